@@ -1,0 +1,173 @@
+"""fp64 CPU oracle for absorbed-form MLA decode (test infrastructure only).
+
+This package is the correctness reference for the GPU library.  Only the test
+suite, the smoke check and the benchmark's CPU-baseline leg may import it; the
+product package never does, and it imports nothing from the product package.
+
+The arithmetic lives in ``mla_oracle.c`` (plain C, IEEE double, OpenMP over
+independent output rows); this module only builds that file and marshals
+arrays.  See the header of ``mla_oracle.c`` for the definition it follows and
+the pages it cites.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "mla_oracle.c")
+LIBRARY = os.path.join(_HERE, "libmla_oracle.so")
+
+D_QK = 576
+D_V = 512
+PAGE = 64
+
+
+def compile_oracle(source: str = SOURCE, output: str = LIBRARY) -> str:
+    """Compile the oracle with gcc (no fast-math: IEEE semantics are kept)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-o", output, source, "-lm"]
+    subprocess.run(cmd, check=True)
+    return output
+
+
+def _needs_build(source: str, output: str) -> bool:
+    return (not os.path.exists(output)
+            or os.path.getmtime(output) < os.path.getmtime(source))
+
+
+class Oracle:
+    """ctypes front end for one compiled copy of the oracle."""
+
+    def __init__(self, library: str = LIBRARY, source: str = SOURCE):
+        if _needs_build(source, library):
+            compile_oracle(source, library)
+        self.path = library
+        self.lib = ctypes.CDLL(library)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        common = [u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int64, ctypes.c_int, ctypes.c_double]
+        for name in ("mla_oracle_direct", "mla_oracle_transposed"):
+            fn = getattr(self.lib, name)
+            fn.argtypes = common + [i32p, ctypes.c_int, f64p, f64p]
+            fn.restype = ctypes.c_int
+        self.lib.mla_oracle_online.argtypes = common + [ctypes.c_int, i32p, ctypes.c_int, f64p, f64p]
+        self.lib.mla_oracle_online.restype = ctypes.c_int
+        self.lib.mla_oracle_split_merge.argtypes = common + [ctypes.c_int, i64p, f64p, f64p]
+        self.lib.mla_oracle_split_merge.restype = ctypes.c_int
+        self.lib.mla_oracle_threads.argtypes = []
+        self.lib.mla_oracle_threads.restype = ctypes.c_int
+
+    # -- marshalling -------------------------------------------------------
+    @staticmethod
+    def _bits(t) -> np.ndarray:
+        """bf16 torch tensor (or uint16 array) -> contiguous uint16 bit array."""
+        if isinstance(t, np.ndarray):
+            assert t.dtype == np.uint16
+            return np.ascontiguousarray(t)
+        import torch
+        assert t.dtype == torch.bfloat16, t.dtype
+        return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+    @staticmethod
+    def _i32(t) -> np.ndarray:
+        if isinstance(t, np.ndarray):
+            return np.ascontiguousarray(t, dtype=np.int32)
+        return np.ascontiguousarray(t.detach().cpu().numpy().astype(np.int32))
+
+    def _common(self, q, kv_cache, block_table, cache_seqlens, scale):
+        qb, kb = self._bits(q), self._bits(kv_cache)
+        bt, sl = self._i32(block_table), self._i32(cache_seqlens)
+        B, s_q, H, dq = qb.shape
+        assert dq == D_QK and kb.shape[1:] == (PAGE, D_QK)
+        assert bt.ndim == 2 and bt.shape[0] == B and sl.shape == (B,)
+        keep = (qb, kb, bt, sl)
+        args = [qb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)),
+                kb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)),
+                bt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                B, s_q, H, kb.shape[0], bt.shape[1], float(scale)]
+        return keep, args, (B, s_q, H)
+
+    @staticmethod
+    def _outputs(B, s_q, H):
+        out = np.full((B, s_q, H, D_V), np.nan, dtype=np.float64)
+        lse = np.full((B, s_q, H), np.nan, dtype=np.float64)
+        return out, lse
+
+    @staticmethod
+    def _seq_list(seqs: Optional[Sequence[int]]):
+        if seqs is None:
+            return None, ctypes.POINTER(ctypes.c_int32)(), 0
+        arr = np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        return arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(arr)
+
+    @staticmethod
+    def _check(rc: int, name: str):
+        if rc != 0:
+            raise ValueError(f"{name} failed with code {rc} "
+                             "(-1 bad argument, -2 block table entry outside the cache, -3 out of memory)")
+
+    # -- the four forms ----------------------------------------------------
+    def direct(self, q, kv_cache, block_table, cache_seqlens, scale, seqs=None):
+        """out[B,s_q,H,512] and lse[B,s_q,H] in float64; rows of sequences not
+        in ``seqs`` (when given) are left as NaN."""
+        keep, args, (B, s_q, H) = self._common(q, kv_cache, block_table, cache_seqlens, scale)
+        out, lse = self._outputs(B, s_q, H)
+        arr, ptr, n = self._seq_list(seqs)
+        rc = self.lib.mla_oracle_direct(*args, ptr, n, _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_direct")
+        return out, lse
+
+    def transposed(self, q, kv_cache, block_table, cache_seqlens, scale, seqs=None):
+        keep, args, (B, s_q, H) = self._common(q, kv_cache, block_table, cache_seqlens, scale)
+        out, lse = self._outputs(B, s_q, H)
+        arr, ptr, n = self._seq_list(seqs)
+        rc = self.lib.mla_oracle_transposed(*args, ptr, n, _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_transposed")
+        return out, lse
+
+    def online(self, q, kv_cache, block_table, cache_seqlens, scale, tile, seqs=None):
+        keep, args, (B, s_q, H) = self._common(q, kv_cache, block_table, cache_seqlens, scale)
+        out, lse = self._outputs(B, s_q, H)
+        arr, ptr, n = self._seq_list(seqs)
+        rc = self.lib.mla_oracle_online(*args, int(tile), ptr, n, _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_online")
+        return out, lse
+
+    def split_merge(self, q, kv_cache, block_table, cache_seqlens, scale, bounds):
+        """``bounds``: int array [B, n_splits + 1] of token boundaries."""
+        keep, args, (B, s_q, H) = self._common(q, kv_cache, block_table, cache_seqlens, scale)
+        bd = np.ascontiguousarray(np.asarray(bounds, dtype=np.int64))
+        assert bd.ndim == 2 and bd.shape[0] == B
+        out, lse = self._outputs(B, s_q, H)
+        rc = self.lib.mla_oracle_split_merge(*args, bd.shape[1] - 1,
+                                             bd.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                             _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_split_merge")
+        return out, lse
+
+    def threads(self) -> int:
+        return int(self.lib.mla_oracle_threads())
+
+
+def _f64(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+_default: Optional[Oracle] = None
+
+
+def default() -> Oracle:
+    """The oracle built from this directory's source (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

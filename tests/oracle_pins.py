@@ -1,0 +1,262 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError on a mismatch.
+They compare against closed forms, library routines (torch's
+scaled_dot_product_attention and logsumexp in float64) and invariants that
+the definition implies -- never against a retyped copy of the oracle's own
+formula.  ``test_oracle.py`` runs them on the oracle;
+``test_oracle_mutants.py`` runs them on copies of the oracle with a planted
+mistake and requires that some pin fails for every mistake.
+
+Source of the definition: the FlashMLA-ETAP explainer (gist.science),
+technical summary, "Methodology / core mechanism" (softmax(Q K^T) V and its
+transposed form), and "FlashMLA: compressing the KV cache" (jsqmd.com),
+"compute flow", step 4 (online softmax).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import mla_inputs as mi
+
+REL = 1e-12
+
+
+def _bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.to(torch.float64).numpy()
+
+
+def _close(a, b, rel=REL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    fin = ~both_inf
+    assert np.all(np.isfinite(a[fin])) and np.all(np.isfinite(b[fin])), what
+    scale = max(1.0, float(np.max(np.abs(b[fin])))) if fin.any() else 1.0
+    err = float(np.max(np.abs(a[fin] - b[fin]))) if fin.any() else 0.0
+    assert err <= rel * scale, f"{what}: max abs err {err:.3e} > {rel * scale:.3e}"
+
+
+def _rows_of(inp: mi.Inputs, b: int, n: int) -> np.ndarray:
+    """Logical cache rows 0..n-1 of sequence b, gathered through the table."""
+    kv = _bf16_to_f64(inp.kv_cache)
+    rows = [kv[int(inp.block_table[b, j // 64]), j % 64] for j in range(n)]
+    return np.stack(rows) if rows else np.zeros((0, 576))
+
+
+# ---------------------------------------------------------------------------
+def pin_single_token(orc):
+    """A one-token context returns that token's value row exactly (its single
+    weight is exp(0) = 1), and lse is the scaled score of that token."""
+    inp = mi.small(B=3, s_q=1, H=4, seqlens=[1, 1, 1], seed=11)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    q = _bf16_to_f64(inp.q)
+    for b in range(3):
+        row = _rows_of(inp, b, 1)[0]
+        for h in range(4):
+            assert np.array_equal(out[b, 0, h], row[:512]), "single token: out != v row"
+            _close(lse[b, 0, h], inp.scale * float(np.dot(q[b, 0, h], row)), what="single token lse")
+
+
+def pin_equal_scores_mean_of_values(orc):
+    """When every key scores the same (query zero on the latent part, keys
+    sharing one rope part), the result is the plain mean of the value rows
+    and lse = s + ln(L)."""
+    L = 77
+    inp = mi.small(B=1, s_q=1, H=2, seqlens=[L], seed=12)
+    inp.q[..., :512] = 0
+    shared_rope = inp.kv_cache[int(inp.block_table[0, 0]), 0, 512:].clone()
+    for j in range(L):
+        inp.kv_cache[int(inp.block_table[0, j // 64]), j % 64, 512:] = shared_rope
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    rows = _rows_of(inp, 0, L)
+    q = _bf16_to_f64(inp.q)
+    for h in range(2):
+        _close(out[0, 0, h], rows[:, :512].mean(axis=0), what="equal scores: mean of V")
+        s = inp.scale * float(np.dot(q[0, 0, h], rows[0]))
+        _close(lse[0, 0, h], s + math.log(L), what="equal scores: lse")
+
+
+def pin_zero_scale(orc):
+    """scale = 0 makes every weight equal: mean of V and lse = ln(n)."""
+    inp = mi.small(B=2, s_q=2, H=2, seqlens=[5, 130], scale=0.0, seed=13)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, 0.0)
+    for b, L in enumerate([5, 130]):
+        for i in range(2):
+            n = L - 1 + i
+            rows = _rows_of(inp, b, n)
+            for h in range(2):
+                _close(out[b, i, h], rows[:, :512].mean(axis=0), what="zero scale: mean")
+                _close(lse[b, i, h], math.log(n), what="zero scale: lse = ln n")
+
+
+def pin_weights_sum_to_one(orc):
+    """Value rows that are all ones give all ones: the weights sum to 1."""
+    inp = mi.small(B=2, s_q=1, H=3, seqlens=[200, 64], seed=14)
+    inp.kv_cache[..., :512] = 1.0
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    assert np.all(np.abs(out - 1.0) <= 1e-14), "constant V: weights do not sum to 1"
+
+
+def pin_two_token_closed_form(orc):
+    """Two tokens with small-integer entries: the scores are exact, and the
+    result is the closed form softmax of two numbers."""
+    inp = mi.small(B=1, s_q=1, H=1, seqlens=[2], table="identity", scale=0.5, seed=15)
+    inp.q.zero_()
+    inp.kv_cache.zero_()
+    inp.q[0, 0, 0, 3] = 2.0       # latent dim 3
+    inp.q[0, 0, 0, 540] = -1.0    # rope dim 540
+    inp.kv_cache[0, 0, 3] = 1.0
+    inp.kv_cache[0, 0, 540] = 3.0
+    inp.kv_cache[0, 0, 7] = 5.0
+    inp.kv_cache[0, 1, 3] = 4.0
+    inp.kv_cache[0, 1, 540] = -2.0
+    inp.kv_cache[0, 1, 7] = -1.0
+    s0 = 0.5 * (2 * 1 + (-1) * 3)    # -0.5
+    s1 = 0.5 * (2 * 4 + (-1) * (-2))  # 5.0
+    e0, e1 = math.exp(s0), math.exp(s1)
+    want = np.zeros(512)
+    want[3] = (e0 * 1 + e1 * 4) / (e0 + e1)
+    want[7] = (e0 * 5 + e1 * -1) / (e0 + e1)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, 0.5)
+    _close(out[0, 0, 0], want, what="two tokens: out")
+    _close(lse[0, 0, 0], math.log(e0 + e1), what="two tokens: lse")
+
+
+def pin_torch_sdpa(orc):
+    """Against torch's scaled_dot_product_attention (float64, CPU) on the
+    gathered rows, query i seeing the first seqlen - s_q + 1 + i rows, with
+    torch.logsumexp for the lse.  Shuffled pages, ragged lengths, s_q = 2."""
+    lens = [1, 63, 64, 65, 130, 300]
+    inp = mi.small(B=len(lens), s_q=2, H=3, seqlens=lens, seed=16)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    q = torch.from_numpy(_bf16_to_f64(inp.q))
+    for b, L in enumerate(lens):
+        rows = torch.from_numpy(_rows_of(inp, b, L))
+        for i in range(2):
+            n = max(0, L - 1 + i)
+            if n == 0:
+                assert np.all(out[b, i] == 0) and np.all(np.isneginf(lse[b, i])), "empty context"
+                continue
+            k = rows[:n].unsqueeze(0)                 # [1, n, 576]
+            v = rows[:n, :512].unsqueeze(0)           # [1, n, 512]
+            qq = q[b, i].unsqueeze(1)                 # [H, 1, 576]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qq, k.expand(3, n, 576), v.expand(3, n, 512), scale=inp.scale)
+            _close(out[b, i], ref[:, 0].numpy(), what=f"sdpa b={b} i={i}")
+            scores = inp.scale * (qq[:, 0] @ rows[:n].T)
+            _close(lse[b, i], torch.logsumexp(scores, dim=-1).numpy(), what=f"lse b={b} i={i}")
+
+
+def pin_causal_rule(orc):
+    """Query 0 of an s_q = 2 call equals an s_q = 1 call on seqlen - 1 tokens
+    with the same query row; query 1 equals an s_q = 1 call on seqlen tokens."""
+    inp = mi.small(B=2, s_q=2, H=2, seqlens=[100, 1], seed=17)
+    out2, lse2 = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    for i, shift in ((0, 1), (1, 0)):
+        q1 = inp.q[:, i:i + 1].clone()
+        lens1 = (inp.cache_seqlens - shift).clamp(min=0)
+        out1, lse1 = orc.direct(q1, inp.kv_cache, inp.block_table, lens1, inp.scale)
+        assert np.array_equal(out1[:, 0], out2[:, i]), f"causal rule, query {i}"
+        assert np.array_equal(lse1[:, 0], lse2[:, i]), f"causal rule lse, query {i}"
+    assert np.all(out2[1, 0] == 0) and np.all(np.isneginf(lse2[1, 0])), "empty context for query 0"
+
+
+def pin_paging_invariance(orc):
+    """The page table only names where rows live: identity and shuffled tables
+    over the same logical rows give bit-identical results."""
+    lens = [65, 190, 7]
+    ident = mi.small(B=3, s_q=1, H=2, seqlens=lens, table="identity", seed=18)
+    shuf = mi.small(B=3, s_q=1, H=2, seqlens=lens, table="shuffled", seed=18)
+    # rebuild the shuffled cache so its logical rows equal the identity cache's
+    kv = torch.empty_like(ident.kv_cache)
+    for b, L in enumerate(lens):
+        for p in range((L + 63) // 64):
+            kv[int(shuf.block_table[b, p])] = ident.kv_cache[int(ident.block_table[b, p])]
+    o1, l1 = orc.direct(ident.q, ident.kv_cache, ident.block_table, ident.cache_seqlens, ident.scale)
+    o2, l2 = orc.direct(ident.q, kv, shuf.block_table, shuf.cache_seqlens, ident.scale)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2), "paging changed the result"
+
+
+def pin_tail_rows_unread(orc):
+    """Cache rows past a sequence's length may hold anything (NaN here)."""
+    lens = [1, 70, 129]
+    clean = mi.small(B=3, s_q=2, H=2, seqlens=lens, seed=19)
+    dirty = mi.small(B=3, s_q=2, H=2, seqlens=lens, seed=19, tail_fill=float("nan"))
+    assert torch.isnan(dirty.kv_cache.float()).any()
+    o1, l1 = orc.direct(clean.q, clean.kv_cache, clean.block_table, clean.cache_seqlens, clean.scale)
+    o2, l2 = orc.direct(dirty.q, dirty.kv_cache, dirty.block_table, dirty.cache_seqlens, dirty.scale)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2), "tail rows reached the result"
+
+
+def pin_transposed_equals_direct(orc):
+    """The method's transposed flow gives the direct flow's result (brute
+    force on tiny inputs)."""
+    for lens, s_q, H in (([1, 3, 8], 1, 4), ([2, 8, 5], 2, 3), ([70, 129], 2, 2)):
+        inp = mi.small(B=len(lens), s_q=s_q, H=H, seqlens=lens, seed=20 + len(lens))
+        a = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+        t = orc.transposed(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+        _close(t[0], a[0], what="transposed out")
+        _close(t[1], a[1], what="transposed lse")
+
+
+def pin_online_equals_direct(orc):
+    """The tiled online-softmax recurrence equals one-shot softmax for any
+    tile size."""
+    lens = [1, 64, 65, 300]
+    inp = mi.small(B=4, s_q=2, H=2, seqlens=lens, seed=24)
+    a = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    for tile in (1, 3, 64, 128, 1000):
+        o = orc.online(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale, tile)
+        _close(o[0], a[0], what=f"online out tile={tile}")
+        _close(o[1], a[1], what=f"online lse tile={tile}")
+
+
+def pin_split_merge_equals_unsplit(orc):
+    """Partial results over token ranges merged through their lse equal the
+    unsplit result, including empty ranges and ranges past the causal limit."""
+    lens = [1, 129, 300]
+    inp = mi.small(B=3, s_q=2, H=2, seqlens=lens, seed=25)
+    a = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    bounds = np.array([[0, 0, 1, 1, 1],
+                       [0, 50, 50, 128, 129],
+                       [0, 1, 150, 299, 300]], dtype=np.int64)
+    m = orc.split_merge(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale, bounds)
+    _close(m[0], a[0], what="split-merge out")
+    _close(m[1], a[1], what="split-merge lse")
+
+
+def pin_outlier_channels(orc):
+    """Outlier latent channels (x20 in q and cache) against SDPA: large logits
+    and near one-hot softmax stay exact in fp64."""
+    inp = mi.small(B=1, s_q=2, H=2, seqlens=[257], outliers=4, seed=26)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    q = torch.from_numpy(_bf16_to_f64(inp.q))
+    rows = torch.from_numpy(_rows_of(inp, 0, 257))
+    for i in range(2):
+        n = 256 + i
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[0, i].unsqueeze(1), rows[:n].unsqueeze(0).expand(2, n, 576),
+            rows[:n, :512].unsqueeze(0).expand(2, n, 512), scale=inp.scale)
+        _close(out[0, i], ref[:, 0].numpy(), rel=1e-11, what="outliers")
+
+
+ALL_PINS = [
+    pin_single_token,
+    pin_equal_scores_mean_of_values,
+    pin_zero_scale,
+    pin_weights_sum_to_one,
+    pin_two_token_closed_form,
+    pin_torch_sdpa,
+    pin_causal_rule,
+    pin_paging_invariance,
+    pin_tail_rows_unread,
+    pin_transposed_equals_direct,
+    pin_online_equals_direct,
+    pin_split_merge_equals_unsplit,
+    pin_outlier_channels,
+]
