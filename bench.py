@@ -1,0 +1,415 @@
+"""Benchmark of absorbed-form MLA decode on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one decode call of the workload through the C ABI: the split-KV
+metadata kernel, the attention kernel and the combine kernel, on inputs that
+are already resident in HBM.  The default workload is the 64K-context,
+16-head configuration (B = 8, s_q = 1, H = 16, L = 65536, 604 MB of cache).
+Between timed steps a 256 MiB buffer (twice the L2) is overwritten outside
+the timed events, so every step starts with a cold L2.
+
+Printed (rank 0, one JSON line): metric / value / unit (microseconds per call,
+lower is better), the attention kernel's roofline against the measured HBM
+copy bandwidth, an end-to-end figure through the same C ABI with the step's
+inputs copied from pinned host memory and its outputs copied back inside the
+timed region, the SM clocks sampled during the timed region, and the fp64
+CPU oracle timed on a bounded sample as a baseline.
+
+With N > 1 (launched by torchrun) every rank runs its own replica of the
+workload on its own GPU (independent batches, no collective on the data
+path); the step time is the max over ranks.  ``--impl reference`` times the
+CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import mla_inputs as mi  # noqa: E402
+
+METRIC = "MLA decode µs/call, achieved HBM TB/s and % roofline at 64K ctx, 16 heads"
+UNIT = "us/call"
+KERNEL_SOURCES = [os.path.join(ROOT, "decode_attention_latent_b200", "csrc", "mla_decode.cu"),
+                  os.path.join(ROOT, "decode_attention_latent_b200", "csrc", "sm100_ptx.cuh")]
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of a per-rank scalar (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        if device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"mla_decode_attention_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m_b or not m_s or m_s.group(1) != source_digest():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 9]
+        os.unlink(self.file.name)
+        samples = []
+        for r in rows:
+            try:
+                ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                samples.append((ts, [x.strip() for x in r]))
+            except Exception:
+                continue
+        inside = [s for ts, s in samples if t0 - 1.0 <= ts <= t1 + 1.0] or [s for _, s in samples]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(s[2]) for s in inside]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in inside:
+            for k, name in enumerate(names):
+                if s[6 + k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(inside[0][3]),
+                "reasons": sorted(reasons), "samples": len(inside),
+                "power_w_max": max(float(s[4]) for s in inside)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample_seconds(orc, inp: mi.Inputs, seqs, tokens: int):
+    """Time the oracle on sequences `seqs`, each truncated to `tokens` tokens."""
+    sub_len = inp.cache_seqlens.clone()
+    sub_len[:] = torch.clamp(sub_len, max=tokens)
+    t0 = time.perf_counter()
+    orc.direct(inp.q, inp.kv_cache, inp.block_table, sub_len, inp.scale, seqs=list(seqs))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp: mi.Inputs, target_s: float = 15.0):
+    """fp64 oracle on a bounded sample of the workload, scaled to one call.
+    The oracle's cost is proportional to (output rows) x (tokens)."""
+    import oracle
+    orc = oracle.default()
+    full_tokens = int(inp.cache_seqlens.max())
+    tokens = min(full_tokens, 4096)
+    t = oracle_sample_seconds(orc, inp, [0], tokens)
+    # grow the sample toward the target: first tokens, then sequences
+    if t > 0 and tokens < full_tokens:
+        tokens = min(full_tokens, max(tokens, int(tokens * (target_s / 2) / t)))
+        t = oracle_sample_seconds(orc, inp, [0], tokens)
+    n_seq = 1
+    if t > 0 and tokens == full_tokens:
+        n_seq = max(1, min(inp.B, int(target_s / t)))
+        if n_seq > 1:
+            t = oracle_sample_seconds(orc, inp, list(range(n_seq)), tokens)
+    work_full = sum(int(x) for x in inp.cache_seqlens)
+    work_sample = n_seq * tokens
+    per_call_s = t * work_full / work_sample
+    return {"value": per_call_s * 1e6, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+            "sample": f"{n_seq} of {inp.B} sequences x {tokens} of {full_tokens} tokens, all "
+                      f"{inp.s_q * inp.H} query rows each, {t:.2f} s, scaled by {work_full / work_sample:.1f}"}
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+    w = mi.WORKLOADS[args.workload]
+    inp = mi.make_inputs(w, seed=0)
+    orc = oracle.default()
+    full_tokens = int(inp.cache_seqlens.max())
+    # each step: sequence 0 truncated so the whole run stays within ~2 minutes
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    tokens = 256
+    t = oracle_sample_seconds(orc, inp, [0], tokens)
+    if t > 0:
+        tokens = int(max(64, min(full_tokens, tokens * per_step / t)))
+    for _ in range(args.warmup):
+        oracle_sample_seconds(orc, inp, [0], tokens)
+    times = [oracle_sample_seconds(orc, inp, [0], tokens) for _ in range(args.steps)]
+    scale = sum(int(x) for x in inp.cache_seqlens) / tokens
+    value = statistics.mean(times) * scale * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "B": w.B, "s_q": w.s_q, "H": w.H,
+                                        "seqlen": w.seqlen, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+                         "sample": f"sequence 0 of {w.B}, first {tokens} of {full_tokens} tokens, "
+                                   f"{w.s_q * w.H} query rows; scaled by {scale:.1f} per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- GPU arm
+def run_ours(args, world, rank, local):
+    import ctypes
+
+    import decode_attention_latent_b200 as mla
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    lib = mla.load_library()
+    w = mi.WORKLOADS[args.workload]
+    inp = mi.make_inputs(w, seed=rank)
+    B, s_q, H = w.B, w.s_q, w.H
+    n_sms = mla.num_sms(dev)
+
+    q = inp.q.to(dev)
+    kv = inp.kv_cache.to(dev)
+    bt = inp.block_table.to(dev)
+    sl = inp.cache_seqlens.to(dev)
+    sched = torch.empty(mla.sched_meta_ints(n_sms), dtype=torch.int32, device=dev)
+    splits = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    ws_bytes = mla.workspace_size(B, s_q, H, n_sms)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(B, s_q, H, mi.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P = ctypes.c_void_p
+
+    def call_metadata():
+        rc = lib.mla_decode_metadata(P(sl.data_ptr()), B, s_q, H, n_sms, P(sched.data_ptr()),
+                                     P(splits.data_ptr()), sp)
+        assert rc == 0, rc
+
+    def call_attention():
+        rc = lib.mla_decode_attention(P(q.data_ptr()), P(kv.data_ptr()), P(bt.data_ptr()), P(sl.data_ptr()),
+                                      B, s_q, H, kv.shape[0], bt.shape[1], ctypes.c_float(inp.scale), n_sms,
+                                      P(sched.data_ptr()), P(splits.data_ptr()), P(ws.data_ptr()), ws_bytes,
+                                      P(out.data_ptr()), P(lse.data_ptr()), sp)
+        assert rc == 0, rc
+
+    def call_combine():
+        rc = lib.mla_decode_combine(P(splits.data_ptr()), P(sched.data_ptr()), P(ws.data_ptr()), ws_bytes,
+                                    B, s_q, H, n_sms, P(out.data_ptr()), P(lse.data_ptr()), sp)
+        assert rc == 0, rc
+
+    # ---- warm-up (untimed)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        call_metadata(); call_attention(); call_combine()
+    torch.cuda.synchronize(dev)
+    assert mla.get_device_error(sched) == 0
+
+    # ---- timed region: K steps, cold L2 at the start of each
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local).start()
+    time.sleep(0.3)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for k in range(K):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream)
+        call_metadata()
+        e[1].record(stream)
+        call_attention()
+        e[2].record(stream)
+        call_combine()
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    meta_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    comb_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    mean_step_ms = max_over_ranks(statistics.mean(step_ms), dev)
+    mean_attn_ms = max_over_ranks(statistics.mean(attn_ms), dev)
+    assert mla.get_device_error(sched) == 0
+
+    # ---- end to end through the C ABI from pinned host buffers
+    q_h = inp.q.pin_memory()
+    bt_h = inp.block_table.pin_memory()
+    sl_h = inp.cache_seqlens.pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    K2 = max(10, K // 4)
+    e2e_ms = []
+    for k in range(K2 + 3):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b_ = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        q.copy_(q_h, non_blocking=True)
+        bt.copy_(bt_h, non_blocking=True)
+        sl.copy_(sl_h, non_blocking=True)
+        call_metadata(); call_attention(); call_combine()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        b_.record(stream)
+        b_.synchronize()
+        if k >= 3:
+            e2e_ms.append(a.elapsed_time(b_))
+    e2e_us = max_over_ranks(statistics.mean(e2e_ms), dev) * 1e3
+
+    # ---- roofline of the attention kernel
+    alg_bytes = mi.algorithmic_bytes(inp)
+    alg_flops = mi.algorithmic_flops(inp)
+    peak, peak_src = measured_peaks()
+    achieved = alg_bytes / (mean_attn_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(args.workload)
+
+    line = {
+        "metric": METRIC,
+        "value": mean_step_ms * 1e3,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": mean_step_ms,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "s_q": s_q, "H": H, "seqlen": w.seqlen,
+                   "page": mi.PAGE, "table": w.table, "kv_bytes": int(inp.kv_cache.numel() * 2),
+                   "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MiB written between steps, outside the events",
+                   "parallelism": f"replicas x{world} (independent batches)", "num_sms": n_sms},
+        "kernels_us": {"metadata": statistics.mean(meta_ms) * 1e3, "attention": statistics.mean(attn_ms) * 1e3,
+                       "combine": statistics.mean(comb_ms) * 1e3},
+        "achieved_tb_s": alg_bytes / (mean_step_ms * 1e-3) / 1e12,
+        "achieved_tflop_s": alg_flops / (mean_step_ms * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "mla_decode_kernel",
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": alg_bytes},
+        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if world > 1:
+        line["aggregate_calls_per_s"] = world / (mean_step_ms * 1e-3)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=mi.HEADLINE, choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

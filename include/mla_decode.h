@@ -1,0 +1,169 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) absorbed-form MLA decode library.
+ *
+ * The operation.  Multi-head latent attention decode over a paged latent KV
+ * cache, in absorbed form: each query head is a 576-wide row (512 latent +
+ * 64 rope columns); each cached token is one 576-wide bf16 row whose first
+ * 512 columns also serve as its value row.  For sequence b, query position
+ * i < s_q and head h:
+ *     n_i  = seqlen_b - s_q + 1 + i            (tokens visible to query i)
+ *     s_j  = softmax_scale * <q[b,i,h,:], k_j>  over j < n_i
+ *     out[b,i,h,:] = sum_j softmax(s)_j * k_j[0:512]          (bf16)
+ *     lse[b,i,h]   = ln(sum_j exp(s_j))                       (fp32)
+ * with out = 0 and lse = -inf when n_i = 0.  This is attention
+ * softmax(Q K^T) V as the FlashMLA-ETAP explainer (gist.science) states it
+ * in its technical summary ("Methodology / core mechanism"), computed the way
+ * that section prescribes: transposed, S^T = K Q^T and O = (V^T P^T)^T, so
+ * that the long KV length fills the matrix-multiply M dimension.  The regime
+ * (1-2 query tokens, 16 heads, 576-wide heads, contexts up to 64K) is the
+ * explainer's "Problem statement" and "Limitations".  The split of the KV
+ * range over many CTAs and the merge through log-sum-exp are the online
+ * softmax of "FlashMLA: compressing the KV cache" (jsqmd.com), "compute
+ * flow", step 4, applied across CTAs instead of across tiles.
+ *
+ * Calls, in the order a decode step makes them:
+ *     mla_decode_metadata   split-KV schedule from the sequence lengths
+ *                           (once per step; reusable by every layer);
+ *     mla_decode            the attention kernel, then the combine kernel;
+ *     mla_decode_attention  the attention kernel alone;
+ *     mla_decode_combine    the combine kernel alone (mla_decode already
+ *                           launches it; exported for tests and timing).
+ *
+ * Conventions for every call.
+ *   - Pointers marked "device" are CUDA device pointers of the current
+ *     device; the caller allocates and owns every buffer, the library
+ *     allocates no device memory and keeps no state between calls.
+ *   - `stream` is a cudaStream_t (0 = the legacy default stream).  All
+ *     launches are asynchronous on it; no call synchronises except
+ *     mla_get_device_error.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE binary32 top
+ *     halves).  Every tensor is dense and row-major with the shape given.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched.  A launch failure returns MLA_ERR_CUDA.  Bad data that only
+ *     the device can see (a page-table entry outside the cache, a length past
+ *     the page table, a schedule built for other shapes, a wait that timed
+ *     out) never traps: the kernel records an MLA_DEVERR_* bit in word 0 of
+ *     sched_meta, skips or substitutes the access, and finishes; read it back
+ *     with mla_get_device_error.
+ *
+ * Supported shapes: s_q in {1, 2}; H in {16, 32, 64, 128}; page size 64;
+ * head widths 576 / 512; 1 <= B <= 4096; 1 <= num_sms <= 4096.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_D_QK 576  /* query / key row width: 512 latent + 64 rope     */
+#define MLA_D_V 512   /* value width: the first 512 columns of a key row  */
+#define MLA_PAGE 64   /* tokens per page of the cache                    */
+#define MLA_TILE 128  /* tokens per attention tile (two pages)           */
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, bad scale */
+    MLA_ERR_MISALIGNED = 2,          /* a pointer breaks its alignment rule    */
+    MLA_ERR_UNSUPPORTED_SHAPE = 3,   /* s_q / H / num_sms outside the set      */
+    MLA_ERR_WORKSPACE_TOO_SMALL = 4, /* workspace_bytes < the required size    */
+    MLA_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed      */
+    MLA_ERR_DEVICE_CHECK = 6         /* mla_get_device_error found a bit set   */
+} mla_status_t;
+
+/* Bits of the device error word (word 0 of sched_meta). */
+#define MLA_DEVERR_BLOCK_TABLE 1   /* page-table entry outside [0, num_blocks)   */
+#define MLA_DEVERR_SEQLEN 2        /* seqlen < 0 or > max_blocks * 64            */
+#define MLA_DEVERR_SCHEDULE 4      /* sched_meta built for other shapes/num_sms  */
+#define MLA_DEVERR_TIMEOUT 8       /* a bounded device-side wait ran out         */
+
+/* Length, in int32 words, of the sched_meta buffer for `num_sms` CTAs. */
+size_t mla_sched_meta_ints(int num_sms);
+
+/* Bytes of workspace mla_decode needs for this shape: fp32 partial outputs and
+ * partial lse of the split-KV pieces.  Returns 0 for an unsupported shape. */
+size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms);
+
+/* Split-KV scheduling metadata.
+ *   cache_seqlens  device int32 [B], tokens cached per sequence.
+ *   num_sms        CTAs the decode will run (normally the SM count, 148 on
+ *                  B200); must equal the value later passed to mla_decode.
+ *   sched_meta     device int32 [mla_sched_meta_ints(num_sms)], written:
+ *                  word 0 = device error word (cleared here), a header
+ *                  describing the shape, then one work range per CTA group.
+ *   num_splits     device int32 [B + 1], written: the prefix sum of the
+ *                  number of pieces each sequence's KV range is cut into
+ *                  (sequence b owns pieces num_splits[b] .. num_splits[b+1]-1).
+ * The KV tiles (128 tokens) of all sequences are laid end to end and cut into
+ * equal contiguous ranges, one per CTA group, so variable lengths balance
+ * across SMs.  Reads the lengths on the device; no host synchronisation. */
+mla_status_t mla_decode_metadata(const int32_t *cache_seqlens, int B, int s_q, int H,
+                                 int num_sms, int32_t *sched_meta, int32_t *num_splits,
+                                 void *stream);
+
+/* The decode.
+ *   q              device bf16 [B, s_q, H, 576], 16-byte aligned.
+ *   kv_cache       device bf16 [num_blocks, 64, 576], 16-byte aligned.
+ *   block_table    device int32 [B, max_blocks]: page p of sequence b lives in
+ *                  kv_cache[block_table[b, p]]; entries past a sequence's
+ *                  last page are never read.
+ *   cache_seqlens  device int32 [B] (the same buffer given to the metadata).
+ *   softmax_scale  finite; applied in fp32 to the scores.
+ *   num_sms, sched_meta, num_splits: exactly as produced by
+ *                  mla_decode_metadata for the same B, s_q, H, lengths.
+ *   workspace      device, 256-byte aligned, workspace_bytes >=
+ *                  mla_decode_workspace_size(B, s_q, H, num_sms).  Scratch
+ *                  only; its contents need no initialisation.
+ *   out            device bf16 [B, s_q, H, 512], 8-byte aligned (written).
+ *   lse            device fp32 [B, s_q, H] (written; natural log).
+ * Launches the attention kernel and then the combine kernel on `stream`. */
+mla_status_t mla_decode(const uint16_t *q, const uint16_t *kv_cache,
+                        const int32_t *block_table, const int32_t *cache_seqlens,
+                        int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                        float softmax_scale, int num_sms,
+                        const int32_t *sched_meta, const int32_t *num_splits,
+                        void *workspace, size_t workspace_bytes,
+                        uint16_t *out, float *lse, void *stream);
+
+/* The attention kernel alone (mla_decode without its combine step), for
+ * callers that schedule the combine themselves or time the kernels apart.
+ * Same arguments and checks as mla_decode.  Rows of one-piece sequences are
+ * final when it returns; the other rows need mla_decode_combine. */
+mla_status_t mla_decode_attention(const uint16_t *q, const uint16_t *kv_cache,
+                                  const int32_t *block_table, const int32_t *cache_seqlens,
+                                  int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                                  float softmax_scale, int num_sms,
+                                  const int32_t *sched_meta, const int32_t *num_splits,
+                                  void *workspace, size_t workspace_bytes,
+                                  uint16_t *out, float *lse, void *stream);
+
+/* The combine kernel alone: for every (b, i, h) whose sequence was cut into
+ * more than one piece, merges the pieces' fp32 partials from the workspace:
+ *     lse = M + ln(sum_k exp(lse_k - M)),  out = sum_k exp(lse_k - lse) * O_k
+ * and writes out (bf16) and lse; rows of sequences with no tokens get
+ * out = 0, lse = -inf; rows of one-piece sequences are left as the decode
+ * wrote them.  Arguments as for mla_decode. */
+mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_meta,
+                                const void *workspace, size_t workspace_bytes,
+                                int B, int s_q, int H, int num_sms,
+                                uint16_t *out, float *lse, void *stream);
+
+/* Waits for `stream`, copies word 0 of sched_meta to *host_code, and returns
+ * MLA_ERR_DEVICE_CHECK if any bit is set (MLA_OK otherwise). */
+mla_status_t mla_get_device_error(const int32_t *sched_meta, int32_t *host_code, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *mla_status_string(mla_status_t status);
+
+/* Text of the last MLA_ERR_CUDA raised on the calling thread (the failing
+ * CUDA call and its error string); "" if none.  Owned by the library. */
+const char *mla_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

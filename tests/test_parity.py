@@ -1,0 +1,231 @@
+"""GPU parity: the sm_100a library (through its C ABI) against the fp64 oracle.
+
+Tolerances (from the arithmetic: bf16 inputs, fp32 accumulation, bf16 P and
+output):
+  out  |gpu - ref| <= 1.5e-2 + |ref| / 256   (1.5e-2 absolute plus one bf16
+       ulp of the reference; for |ref| < 0.6 this is the plain 1.5e-2 bound)
+       and relative RMSE  sqrt(sum (gpu-ref)^2 / sum ref^2) <= 5e-3;
+  lse  |gpu - ref| <= 1e-3, and -inf exactly where the reference is -inf.
+Integer work (the schedule) is compared exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_latent_b200 as mla
+import mla_inputs as mi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 1.5e-2
+RTOL = 1.0 / 256.0
+RMSE_MAX = 5e-3
+LSE_ATOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    mla.load_library()
+    return torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+def run_gpu(inp: mi.Inputs, dev, n_sms=None, q=None):
+    qd = (inp.q if q is None else q).to(dev)
+    kv = inp.kv_cache.to(dev)
+    bt = inp.block_table.to(dev)
+    sl = inp.cache_seqlens.to(dev)
+    n = mla.num_sms(dev) if n_sms is None else n_sms
+    sched, splits = mla.decode_metadata(sl, inp.s_q, inp.H, n)
+    out, lse = mla.decode(qd, kv, bt, sl, inp.scale, sched_meta=sched, num_splits=splits, num_sms_=n)
+    err = mla.get_device_error(sched)
+    return out.float().cpu().numpy(), lse.cpu().numpy(), err, sched, splits
+
+
+def compare(g_out, g_lse, r_out, r_lse, seqs=None, what=""):
+    if seqs is not None:
+        g_out, g_lse, r_out, r_lse = g_out[seqs], g_lse[seqs], r_out[seqs], r_lse[seqs]
+    fin = np.isfinite(r_lse)
+    assert np.array_equal(np.isfinite(g_lse), fin), f"{what}: lse finiteness differs"
+    assert np.all(g_lse[~fin] == -np.inf), f"{what}: empty rows must have lse = -inf"
+    assert np.all(g_out[~fin] == 0), f"{what}: empty rows must have out = 0"
+    err = np.abs(g_out - r_out)
+    bound = ATOL + RTOL * np.abs(r_out)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert np.all(err <= bound), (f"{what}: out err {err[worst]:.4e} > {bound[worst]:.4e} at {worst} "
+                                  f"(gpu {g_out[worst]:.6f} ref {r_out[worst]:.6f})")
+    den = float(np.sum(r_out.astype(np.float64) ** 2))
+    if den > 0:
+        rmse = math.sqrt(float(np.sum((g_out - r_out) ** 2)) / den)
+        assert rmse <= RMSE_MAX, f"{what}: relative RMSE {rmse:.3e}"
+    if fin.any():
+        lerr = np.abs(g_lse[fin] - r_lse[fin])
+        assert lerr.max() <= LSE_ATOL, f"{what}: lse err {lerr.max():.3e}"
+    return float(err.max())
+
+
+# -------------------------------------------------------------- workloads
+SAMPLED = {  # sequences the oracle checks at full size
+    "b1_h16_l1k_identity": None,
+    "b16_h16_l4k": None,
+    "b32_sq2_h16_l16k_outliers": [0, 13, 31],
+    "b64_h128_lvar1k32k": [0, 7, 33, 63],
+    "b8_h16_l64k": [0, 5],
+}
+
+
+@pytest.mark.parametrize("name", list(mi.WORKLOADS))
+def test_workload_parity(dev, orc, name):
+    inp = mi.make_inputs(mi.WORKLOADS[name], seed=0)
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev)
+    assert err == 0, f"device error word {err}"
+    seqs = SAMPLED[name]
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale, seqs=seqs)
+    compare(g_out, g_lse, r_out, r_lse, seqs=seqs, what=name)
+
+
+# ------------------------------------------------------------ edge cases
+RAGGED = [1, 63, 64, 65, 127, 128, 129, 1000]
+
+
+@pytest.mark.parametrize("s_q,H", [(1, 16), (1, 32), (1, 64), (1, 128), (2, 16), (2, 32), (2, 64), (2, 128)])
+def test_ragged_lengths_all_shapes(dev, orc, s_q, H):
+    inp = mi.small(B=len(RAGGED), s_q=s_q, H=H, seqlens=RAGGED, seed=100 + H + s_q, tail_fill=float("nan"))
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev)
+    assert err == 0
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"ragged s_q={s_q} H={H}")
+
+
+@pytest.mark.parametrize("n_sms", [1, 2, 3, 17, 148, 400])
+def test_forced_split_counts(dev, orc, n_sms):
+    lens = [5, 700, 129, 2048, 64]
+    inp = mi.small(B=len(lens), s_q=2, H=16, seqlens=lens, seed=200, tail_fill=float("nan"))
+    g_out, g_lse, err, _, splits = run_gpu(inp, dev, n_sms=n_sms)
+    assert err == 0
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"num_sms={n_sms}")
+
+
+def test_empty_sequences(dev, orc):
+    lens = [0, 300, 0, 1]
+    inp = mi.small(B=4, s_q=2, H=16, seqlens=lens, seed=300)
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev, n_sms=7)
+    assert err == 0
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what="empty sequences")
+
+
+def test_identity_and_shuffled_tables_bitwise(dev):
+    lens = [4096, 1000, 129]
+    ident = mi.small(B=3, s_q=1, H=16, seqlens=lens, table="identity", seed=400)
+    shuf = mi.small(B=3, s_q=1, H=16, seqlens=lens, table="shuffled", seed=400)
+    kv = torch.empty_like(ident.kv_cache)
+    for b, L in enumerate(lens):
+        for p in range(mi.pages_for(L)):
+            kv[int(shuf.block_table[b, p])] = ident.kv_cache[int(ident.block_table[b, p])]
+    shuf.kv_cache = kv
+    a = run_gpu(ident, dev)
+    b = run_gpu(shuf, dev)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]), "page table changed the result"
+
+
+def test_repeat_runs_bitwise(dev):
+    inp = mi.small(B=4, s_q=2, H=16, seqlens=[3000, 17, 640, 2500], seed=500)
+    a = run_gpu(inp, dev)
+    b = run_gpu(inp, dev)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_head_permutation(dev):
+    inp = mi.small(B=2, s_q=1, H=32, seqlens=[900, 2100], seed=600)
+    perm = torch.randperm(32, generator=torch.Generator().manual_seed(1))
+    a = run_gpu(inp, dev)
+    b = run_gpu(inp, dev, q=inp.q[:, :, perm].contiguous())
+    np.testing.assert_allclose(b[0], a[0][:, :, perm.numpy()], rtol=0, atol=1e-2)
+    np.testing.assert_allclose(b[1], a[1][:, :, perm.numpy()], rtol=0, atol=1e-4)
+
+
+def test_causal_query0_matches_shorter_context(dev):
+    inp = mi.small(B=3, s_q=2, H=16, seqlens=[1, 130, 4000], seed=700)
+    two = run_gpu(inp, dev)
+    one = mi.Inputs(q=inp.q[:, :1].contiguous(), kv_cache=inp.kv_cache, block_table=inp.block_table,
+                    cache_seqlens=(inp.cache_seqlens - 1).clamp(min=0), scale=inp.scale)
+    single = run_gpu(one, dev)
+    compare(two[0][:, :1], two[1][:, :1], single[0].astype(np.float64), single[1].astype(np.float64),
+            what="query 0 vs shorter context")
+
+
+def test_bad_block_table_sets_error_word(dev):
+    inp = mi.small(B=2, s_q=1, H=16, seqlens=[300, 200], seed=800)
+    inp.block_table[1, 2] = inp.kv_cache.shape[0] + 5  # outside the cache
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev)
+    assert err & mla.DEVERR_BLOCK_TABLE
+    assert np.all(np.isfinite(g_out[0]))  # the other sequence is untouched by the bad entry
+
+
+def test_schedule_for_other_shape_is_detected(dev):
+    inp = mi.small(B=2, s_q=1, H=16, seqlens=[300, 200], seed=801)
+    sl = inp.cache_seqlens.to(dev)
+    sched, splits = mla.decode_metadata(sl, 1, 32, 16)  # built for H=32
+    out, lse = mla.decode(inp.q.to(dev), inp.kv_cache.to(dev), inp.block_table.to(dev), sl, inp.scale,
+                          sched_meta=sched, num_splits=splits, num_sms_=16)
+    assert mla.get_device_error(sched) & mla.DEVERR_SCHEDULE
+
+
+# ---------------------------------------------------- schedule (integers)
+def expected_schedule(lens, tuples):
+    tiles = [(max(0, L) + 127) // 128 for L in lens]
+    prefix = np.concatenate([[0], np.cumsum(tiles)]).astype(int)
+    total = int(prefix[-1])
+    per = max(1, -(-total // tuples)) if total else 1
+    owner = {}  # (b, tile) -> tuple
+    for k in range(tuples):
+        for f in range(k * per, min((k + 1) * per, total)):
+            b = int(np.searchsorted(prefix, f, side="right") - 1)
+            owner[(b, f - int(prefix[b]))] = k
+    nsplit = []
+    for b, nt in enumerate(tiles):
+        nsplit.append(len({owner[(b, t)] for t in range(nt)}))
+    return owner, np.concatenate([[0], np.cumsum(nsplit)]).astype(int)
+
+
+@pytest.mark.parametrize("lens,n_sms,H", [
+    ([65536] * 8, 148, 16), ([5, 700, 129, 2048, 64], 17, 16), ([0, 300, 0, 1], 7, 16),
+    (list(range(1, 4000, 97)), 148, 128), ([1024] * 3, 400, 32),
+])
+def test_metadata_matches_partition_rule(dev, lens, n_sms, H):
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    sched, splits = mla.decode_metadata(sl, 1, H, n_sms)
+    G = max(1, H // 64)
+    tuples = n_sms // G
+    owner, base = expected_schedule(lens, tuples)
+    assert np.array_equal(splits.cpu().numpy(), base)
+    s = sched.cpu().numpy()
+    assert s[0] == 0
+    seen = {}
+    for k in range(tuples):
+        b0, t0, b1, t1, sp0 = s[16 + 8 * k: 16 + 8 * k + 5]
+        if b0 < 0:
+            continue
+        for b in range(b0, b1 + 1):
+            nt = (lens[b] + 127) // 128
+            tb = t0 if b == b0 else 0
+            te = t1 if b == b1 else nt
+            for t in range(tb, te):
+                assert (b, t) not in seen
+                seen[(b, t)] = k
+            if tb < te:
+                piece = sp0 if b == b0 else 0
+                first_owner = min(v for (bb, _), v in owner.items() if bb == b)
+                assert piece == k - first_owner
+    assert seen == owner
