@@ -40,7 +40,8 @@ DEVERR_TIMEOUT = 8
 
 EXPORTED = (
     "mla_sched_meta_ints", "mla_decode_workspace_size", "mla_decode_metadata",
-    "mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_get_device_error",
+    "mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_static_workspace",
+    "mla_get_device_error",
     "mla_status_string", "mla_last_error_message",
 )
 
@@ -81,6 +82,9 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
     lib.mla_decode.restype = ci
     lib.mla_decode_attention.argtypes = lib.mla_decode.argtypes
     lib.mla_decode_attention.restype = ci
+    lib.mla_decode_static_workspace.argtypes = [cu16p, cu16p, i32p, i32p, ci, ci, ci, ctypes.c_int64, ci,
+                                                ctypes.c_float, ci, i32p, i32p, cu16p, vp, vp]
+    lib.mla_decode_static_workspace.restype = ci
     lib.mla_decode_combine.argtypes = [i32p, i32p, vp, sz, ci, ci, ci, ci, cu16p, vp, vp]
     lib.mla_decode_combine.restype = ci
     lib.mla_get_device_error.argtypes = [i32p, ctypes.POINTER(ctypes.c_int32), vp]

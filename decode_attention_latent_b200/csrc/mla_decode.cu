@@ -1536,6 +1536,41 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
 }  // namespace host
 }  // namespace mla
 
+// Scratch for callers that cannot allocate device memory: a fixed, file-scope
+// device array that lives as long as the library is loaded.  Host code must not
+// pass the array's name to a kernel (on the host it is only a stand-in); it
+// passes the device address that cudaGetSymbolAddress returns for the current
+// device.
+static __device__ __align__(256) unsigned char g_static_workspace[MLA_STATIC_WORKSPACE_BYTES];
+
+namespace mla {
+namespace host {
+
+std::mutex g_static_ws_mutex;
+void *g_static_ws_ptr[64] = {nullptr};
+
+// Device address of g_static_workspace on the current device, resolved once
+// per device (the first call on a device does this; it makes no allocation).
+mla_status_t static_workspace_address(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return cuda_fail(cudaErrorInvalidDevice, "device index");
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_workspace);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+        g_static_ws_ptr[dev] = ptr;
+    }
+    *out = g_static_ws_ptr[dev];
+    return MLA_OK;
+}
+
+}  // namespace host
+}  // namespace mla
+
 using namespace mla;
 using namespace mla::host;
 
@@ -1706,6 +1741,30 @@ mla_status_t mla_decode(const uint16_t *q, const uint16_t *kv_cache, const int32
     if (rc != MLA_OK) return rc;
     return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
                               stream);
+}
+
+mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_cache, const int32_t *block_table,
+                                         const int32_t *cache_seqlens, int B, int s_q, int H, int64_t num_blocks,
+                                         int max_blocks, float softmax_scale, int num_sms,
+                                         const int32_t *sched_meta, const int32_t *num_splits, uint16_t *out,
+                                         float *lse, void *stream)
+{
+    const size_t need = mla_decode_workspace_size(B, s_q, H, num_sms);
+    if (need == 0) {
+        if (B < 1 || B > kMaxBatch) return MLA_ERR_INVALID_ARG;
+        return MLA_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (need > MLA_STATIC_WORKSPACE_BYTES) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "mla_decode_static_workspace: this shape needs %zu bytes of workspace, the built-in one holds %zu",
+                 need, static_cast<size_t>(MLA_STATIC_WORKSPACE_BYTES));
+        return MLA_ERR_WORKSPACE_TOO_SMALL;
+    }
+    void *ws = nullptr;
+    const mla_status_t rc = static_workspace_address(&ws);
+    if (rc != MLA_OK) return rc;
+    return mla_decode(q, kv_cache, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks, softmax_scale,
+                      num_sms, sched_meta, num_splits, ws, MLA_STATIC_WORKSPACE_BYTES, out, lse, stream);
 }
 
 mla_status_t mla_get_device_error(const int32_t *sched_meta, int32_t *host_code, void *stream)

@@ -151,6 +151,40 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
                                 int B, int s_q, int H, int num_sms,
                                 uint16_t *out, float *lse, void *stream);
 
+/* Size of the workspace built into the library for mla_decode_static_workspace. */
+#define MLA_STATIC_WORKSPACE_BYTES (8u << 20)
+
+/* mla_decode without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code that runs where device allocation is not
+ * permitted or not wanted -- a host application whose device memory is
+ * reserved up front by its own pool, or a plugin inside a framework that owns
+ * every allocation -- and so cannot obtain the scratch buffer mla_decode
+ * expects.  The scratch is a fixed device array compiled into the library
+ * (MLA_STATIC_WORKSPACE_BYTES, 8 MiB); every GPU that loads the library holds
+ * it until the process exits.  The paper has no counterpart: this is a
+ * packaging convenience, not part of the method.
+ *
+ * Arguments, layouts and results are those of mla_decode without `workspace`
+ * and `workspace_bytes`; the caller still passes every input and output.  This
+ * call makes no device allocation and frees nothing.
+ *   - Returns MLA_ERR_WORKSPACE_TOO_SMALL, without launching, when the shape
+ *     needs more than MLA_STATIC_WORKSPACE_BYTES
+ *     (mla_decode_workspace_size(B, s_q, H, num_sms) tells); the message is in
+ *     mla_last_error_message.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (once; no allocation).  Make that first call before capturing any
+ *     stream.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (every value read is written first
+ *     by the same call), but calls whose kernels overlap on the GPU -- on two
+ *     streams, or from two host threads -- race on it: serialise them. */
+mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_cache,
+                                         const int32_t *block_table, const int32_t *cache_seqlens,
+                                         int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                                         float softmax_scale, int num_sms,
+                                         const int32_t *sched_meta, const int32_t *num_splits,
+                                         uint16_t *out, float *lse, void *stream);
+
 /* Waits for `stream`, copies word 0 of sched_meta to *host_code, and returns
  * MLA_ERR_DEVICE_CHECK if any bit is set (MLA_OK otherwise). */
 mla_status_t mla_get_device_error(const int32_t *sched_meta, int32_t *host_code, void *stream);
