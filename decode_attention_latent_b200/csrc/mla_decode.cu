@@ -162,7 +162,7 @@ __device__ __forceinline__ float warp_sum(float x)
 // flattened tiles [k * per, min((k + 1) * per, total)).  Sequence b is cut
 // into one piece per group whose range meets it; those pieces are numbered
 // from split_base[b].
-constexpr int kMetaThreads = 1024;
+constexpr int kMetaThreads = 128;
 
 __device__ int block_exclusive_scan(int *arr, int n, int *warp_sums)
 {
@@ -183,7 +183,7 @@ __device__ int block_exclusive_scan(int *arr, int n, int *warp_sums)
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_sums[lane];
+        int w = lane < kMetaThreads / 32 ? warp_sums[lane] : 0;  // lanes past the last warp add nothing
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -1283,6 +1283,7 @@ mla_decode_ss_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_co
     Smem sm;
     Range w;
     uint32_t tmem;
+    ptx::griddep_launch_dependents();
     if (!decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) return;
     const int warp = threadIdx.x >> 5;
     const int g = blockIdx.x % p.G;
@@ -1301,6 +1302,7 @@ mla_decode_tv_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_co
     Smem sm;
     Range w;
     uint32_t tmem;
+    ptx::griddep_launch_dependents();
     if (!decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) return;
     const int warp = threadIdx.x >> 5;
     const int g = blockIdx.x % p.G;
@@ -1313,75 +1315,86 @@ mla_decode_tv_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_co
 }
 
 // =============================================================== combine
-constexpr int kCombineWarps = 8;
+// One 128-thread block per output row (b, i, h) of a sequence cut into pieces.
+// The pieces' lse values go to shared memory once; each thread then owns four
+// latent dims and issues its loads of every piece unrolled, so the partials
+// (fresh in L2) are fetched with all loads in flight instead of one piece at a
+// time.  Launched as a programmatic dependent of the attention kernel: it may
+// become resident early and waits in hardware for that grid to finish.
+constexpr int kCombineThreads = 128;
 
-__global__ void __launch_bounds__(kCombineWarps * 32)
+__global__ void __launch_bounds__(kCombineThreads)
 mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restrict__ ws_o,
                    const float *__restrict__ ws_lse, int B, int s_q, int H, int HG, int G, int max_pieces,
                    uint16_t *__restrict__ out, float *__restrict__ lse, int32_t *__restrict__ err)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t r = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
-    if (r >= static_cast<int64_t>(B) * s_q * H) return;
+    constexpr int kBatch = 16;  // pieces whose loads are in flight together
+    ptx::griddep_wait();        // the attention grid (and its memory) is complete
+    const int tid = threadIdx.x;
+    const int64_t r = blockIdx.x;
     const int h = static_cast<int>(r % H);
     const int i = static_cast<int>((r / H) % s_q);
     const int b = static_cast<int>(r / (static_cast<int64_t>(H) * s_q));
     const int first = split_base[b];
     const int n = split_base[b + 1] - first;
-    if (n == 1) return;  // written directly by the decode kernel
-    uint16_t *o = out + r * kDV;
+    if (n == 1) return;  // written directly by the attention kernel
+    uint2 *o = reinterpret_cast<uint2 *>(out + r * kDV) + tid;  // four bf16 per thread
     if (n <= 0) {
-        for (int d = lane; d < kDV; d += 32) o[d] = 0;
-        if (lane == 0) lse[r] = -INFINITY;
+        *o = make_uint2(0, 0);
+        if (tid == 0) lse[r] = -INFINITY;
         return;
     }
-    if (first < 0 || (static_cast<int64_t>(first) + n) * G > max_pieces) {
-        if (lane == 0) atomicOr(err, MLA_DEVERR_SCHEDULE);
+    if (first < 0 || (static_cast<int64_t>(first) + n) * G > max_pieces || n > kMaxSms) {
+        if (tid == 0) atomicOr(err, MLA_DEVERR_SCHEDULE);
         return;
     }
     const int g = h / HG, hl = h % HG;
-    auto piece_row = [&](int k) -> int64_t {
-        return (static_cast<int64_t>(first + k) * G + g) * s_q * HG + static_cast<int64_t>(i) * HG + hl;
-    };
+    const int64_t row0 = (static_cast<int64_t>(first) * G + g) * s_q * HG + static_cast<int64_t>(i) * HG + hl;
+    const int64_t pstride = static_cast<int64_t>(G) * s_q * HG;  // rows between consecutive pieces
+    const float *lsrc = ws_lse + row0;
+    const float4 *src = reinterpret_cast<const float4 *>(ws_o + row0 * kDV) + tid;
+    const int64_t step = pstride * kDV / 4;  // float4s between consecutive pieces
+    // Every thread reads all piece lse values itself (broadcast loads) together
+    // with its own partials, so the merge costs one round trip per batch.
     float M = -INFINITY;
-    for (int k = lane; k < n; k += 32) M = fmaxf(M, ws_lse[piece_row(k)]);
-    M = warp_max(M);
-    if (M == -INFINITY) {
-        for (int d = lane; d < kDV; d += 32) o[d] = 0;
-        if (lane == 0) lse[r] = -INFINITY;
+    for (int k = 0; k < n; ++k) M = fmaxf(M, lsrc[k * pstride]);
+    if (M == -INFINITY) {  // every piece saw no token
+        *o = make_uint2(0, 0);
+        if (tid == 0) lse[r] = -INFINITY;
         return;
     }
-    float s = 0.f;
-    for (int k = lane; k < n; k += 32) s += expf(ws_lse[piece_row(k)] - M);
-    s = warp_sum(s);
-    const float total = M + logf(s);
-    float4 acc[4];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ssum = 0.f;
+    for (int k0 = 0; k0 < n; k0 += kBatch) {
+        float4 x[kBatch];
+        float lk[kBatch];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < n; ++k) {
-        const int64_t pr = piece_row(k);
-        const float wk = expf(ws_lse[pr] - total);
-        const float4 *src = reinterpret_cast<const float4 *>(ws_o + pr * kDV);
+        for (int u = 0; u < kBatch; ++u) {
+            if (k0 + u < n) {
+                x[u] = src[(k0 + u) * step];
+                lk[u] = lsrc[(k0 + u) * pstride];
+            }
+        }
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const float4 x = src[v * 32 + lane];
-            acc[v].x += wk * x.x;
-            acc[v].y += wk * x.y;
-            acc[v].z += wk * x.z;
-            acc[v].w += wk * x.w;
+        for (int u = 0; u < kBatch; ++u) {
+            if (k0 + u < n) {
+                const float wk = expf(lk[u] - M);
+                ssum += wk;
+                acc.x += wk * x[u].x;
+                acc.y += wk * x[u].y;
+                acc.z += wk * x[u].z;
+                acc.w += wk * x[u].w;
+            }
         }
     }
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const int d = (v * 32 + lane) * 4;
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[v].x, acc[v].y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[v].z, acc[v].w);
-        uint2 packed;
-        packed.x = *reinterpret_cast<uint32_t *>(&lo);
-        packed.y = *reinterpret_cast<uint32_t *>(&hi);
-        *reinterpret_cast<uint2 *>(o + d) = packed;
-    }
-    if (lane == 0) lse[r] = total;
+    const float inv = 1.f / ssum;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t *>(&lo);
+    packed.y = *reinterpret_cast<uint32_t *>(&hi);
+    *o = packed;
+    if (tid == 0) lse[r] = M + logf(ssum);
 }
 
 // ================================================================== host
@@ -1627,11 +1640,18 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
     const float *ws_o = static_cast<const float *>(workspace);
     const float *ws_lse = reinterpret_cast<const float *>(static_cast<const char *>(workspace) + wl.lse_off);
     const int64_t rows = static_cast<int64_t>(B) * s_q * H;
-    const int grid = static_cast<int>((rows + kCombineWarps - 1) / kCombineWarps);
-    mla_combine_kernel<<<grid, kCombineWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
-        num_splits, ws_o, ws_lse, B, s_q, H, sh.HG, sh.G, wl.pieces, out, lse,
-        const_cast<int32_t *>(sched_meta));
-    const cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mla_combine_kernel, num_splits, ws_o, ws_lse, B, s_q, H, sh.HG, sh.G,
+                                       wl.pieces, out, lse, const_cast<int32_t *>(sched_meta));
     if (e != cudaSuccess) return cuda_fail(e, "mla_combine_kernel launch");
     return MLA_OK;
 }

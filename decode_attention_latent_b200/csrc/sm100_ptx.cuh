@@ -333,6 +333,16 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
     return r != 0;
 }
 
+// Programmatic dependent launch: let the next kernel of the stream start
+// launching, and (in that kernel) wait until the previous grid has completed
+// and its memory operations are visible.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns()
 {
     uint64_t t;

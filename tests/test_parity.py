@@ -202,6 +202,7 @@ def expected_schedule(lens, tuples):
 @pytest.mark.parametrize("lens,n_sms,H", [
     ([65536] * 8, 148, 16), ([5, 700, 129, 2048, 64], 17, 16), ([0, 300, 0, 1], 7, 16),
     (list(range(1, 4000, 97)), 148, 128), ([1024] * 3, 400, 32),
+    ([int(x) for x in np.random.default_rng(5).integers(0, 3000, 4096)], 148, 16),
 ])
 def test_metadata_matches_partition_rule(dev, lens, n_sms, H):
     sl = torch.tensor(lens, dtype=torch.int32, device=dev)
