@@ -49,7 +49,15 @@ UNIT = "us/call"
 KERNEL_SOURCES = [os.path.join(ROOT, "decode_attention_latent_b200", "csrc", "mla_decode.cu"),
                   os.path.join(ROOT, "decode_attention_latent_b200", "csrc", "sm100_ptx.cuh")]
 FALLBACK_HBM_GBS = 6650.0
-KV_COPIES = 2  # consecutive steps read different copies of the cache
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 << 20
+
+
+def kv_copy_count(kv_bytes: int, l2_bytes: int) -> int:
+    """Device copies of the cache that consecutive steps cycle through: at
+    least two, and enough that a step's cache was last read at least three
+    L2 capacities of traffic earlier (so it cannot be found in L2)."""
+    return max(2, -(-3 * l2_bytes // max(1, kv_bytes)))
 
 
 # ---------------------------------------------------------------- helpers
@@ -83,13 +91,40 @@ def barrier(device):
 
 
 def measured_peaks():
+    """(HBM GB/s, its source, bf16 TFLOP/s burst, its source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+        return (float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)",
+                float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)")
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+        return (FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)",
+                FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s earlier pool measurement)")
+
+
+def attention_kernel_name(s_q: int, H: int) -> str:
+    """The attention kernel the library launches for this shape: N = s_q * H
+    query columns per CTA (64 at most); N <= 32 keeps V^T in TMEM."""
+    return "mla_decode_tv_kernel" if min(s_q * H, 64) <= 32 else "mla_decode_ss_kernel"
+
+
+def roofline(alg_bytes: int, alg_flops: int, seconds: float, peaks) -> dict:
+    """Roofline of one attention launch: the bound is whichever of the HBM
+    time (algorithmic bytes / copy bandwidth) and the tensor time
+    (algorithmic FLOPs / bf16 GEMM peak) is longer."""
+    hbm, hbm_src, tc, tc_src = peaks
+    t_hbm = alg_bytes / (hbm * 1e9)
+    t_tc = alg_flops / (tc * 1e12)
+    both = {"hbm_frac": t_hbm / seconds, "tensor_frac": t_tc / seconds,
+            "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}
+    if t_tc > t_hbm:
+        a = alg_flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": tc, "unit": "TFLOP/s", "frac": a / tc,
+                "peak_source": tc_src, "both": both}
+    a = alg_bytes / seconds / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+            "peak_source": hbm_src, "both": both}
 
 
 def source_digest() -> str:
@@ -255,7 +290,10 @@ def run_ours(args, world, rank, local):
     n_sms = mla.num_sms(dev)
 
     q = inp.q.to(dev)
-    kv_copies = [inp.kv_cache.to(dev) for _ in range(KV_COPIES)]
+    kv_bytes = int(inp.kv_cache.numel() * 2)
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", L2_BYTES) or L2_BYTES)
+    n_copies = kv_copy_count(kv_bytes, l2)
+    kv_copies = [inp.kv_cache.to(dev) for _ in range(n_copies)]
     kv = kv_copies[0]
     bt = inp.block_table.to(dev)
     sl = inp.cache_seqlens.to(dev)
@@ -288,7 +326,7 @@ def run_ours(args, world, rank, local):
 
     # ---- warm-up (untimed)
     for k in range(max(3, args.warmup)):
-        call_metadata(); call_attention(kv_copies[k % KV_COPIES]); call_combine()
+        call_metadata(); call_attention(kv_copies[k % n_copies]); call_combine()
     torch.cuda.synchronize(dev)
     assert mla.get_device_error(sched) == 0
 
@@ -306,7 +344,7 @@ def run_ours(args, world, rank, local):
         e[0].record(stream)
         call_metadata()
         e[1].record(stream)
-        call_attention(kv_copies[k % KV_COPIES])
+        call_attention(kv_copies[k % n_copies])
         e[2].record(stream)
         call_combine()
         e[3].record(stream)
@@ -326,7 +364,7 @@ def run_ours(args, world, rank, local):
         e = ev2[k]
         e[0].record(stream)
         call_metadata()
-        call_attention(kv_copies[k % KV_COPIES])
+        call_attention(kv_copies[k % n_copies])
         call_combine()
         e[1].record(stream)
     torch.cuda.synchronize(dev)
@@ -354,7 +392,7 @@ def run_ours(args, world, rank, local):
         q.copy_(q_h, non_blocking=True)
         bt.copy_(bt_h, non_blocking=True)
         sl.copy_(sl_h, non_blocking=True)
-        call_metadata(); call_attention(kv_copies[k % KV_COPIES]); call_combine()
+        call_metadata(); call_attention(kv_copies[k % n_copies]); call_combine()
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
         b_.record(stream)
@@ -366,9 +404,11 @@ def run_ours(args, world, rank, local):
     # ---- roofline of the attention kernel
     alg_bytes = mi.algorithmic_bytes(inp)
     alg_flops = mi.algorithmic_flops(inp)
-    peak, peak_src = measured_peaks()
-    achieved = alg_bytes / (mean_attn_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(args.workload)
+    roof = roofline(alg_bytes, alg_flops, mean_attn_ms * 1e-3, measured_peaks())
+    roof["traffic"] = ncu_traffic(args.workload)
+    roof["kernel"] = attention_kernel_name(s_q, H)
+    roof["algorithmic_bytes_per_launch"] = alg_bytes
+    roof["algorithmic_flops_per_launch"] = alg_flops
 
     line = {
         "metric": METRIC,
@@ -385,15 +425,13 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": args.workload, "B": B, "s_q": s_q, "H": H, "seqlen": w.seqlen,
                    "page": mi.PAGE, "table": w.table, "kv_bytes": int(inp.kv_cache.numel() * 2),
-                   "l2": f"inputs larger than L2: {KV_COPIES} device copies of the {int(inp.kv_cache.numel() * 2) >> 20} MiB cache, alternated step by step; no flush",
+                   "l2": f"inputs larger than L2: {n_copies} device copies of the {kv_bytes / 2**20:.1f} MiB cache, used in turn step by step ({n_copies * kv_bytes / l2:.1f}x the {l2 >> 20} MiB L2); no flush",
                    "parallelism": f"replicas x{world} (independent batches)", "num_sms": n_sms},
         "kernels_us": {"metadata": statistics.mean(meta_ms) * 1e3, "attention": statistics.mean(attn_ms) * 1e3,
                        "combine": statistics.mean(comb_ms) * 1e3},
         "achieved_tb_s": alg_bytes / (mean_step_ms * 1e-3) / 1e12,
         "achieved_tflop_s": alg_flops / (mean_step_ms * 1e-3) / 1e12,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "kernel": "mla_decode_kernel",
-                     "peak_source": peak_src, "algorithmic_bytes_per_launch": alg_bytes},
+        "roofline": roof,
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * K,
         "timing": "value/ms_per_step: events around whole steps (region 2); kernels_us and roofline: events between kernels (region 1)",

@@ -5,7 +5,7 @@
 //   mla_metadata_kernel  split-KV schedule: the 128-token tiles of all
 //                        sequences are laid end to end and cut into equal
 //                        contiguous ranges, one per CTA group.
-//   mla_decode_*_kernel  one persistent CTA per SM.  Per 128-token tile:
+//   mla_decode_kernel    one persistent CTA per SM.  Per 128-token tile:
 //                          TMA gathers the tile's two pages through the page
 //                          table into a ring of 16 KB shared-memory slots
 //                          (one slot = 64 columns of 128 rows, 128-byte
@@ -28,19 +28,13 @@
 //                        softmax of "FlashMLA: compressing the KV cache",
 //                        jsqmd.com, "compute flow" step 4, across CTAs).
 //
-// Two variants of the attention kernel:
-//
-//   tv (N <= 32)  The V part of each tile is copied, transposed, from its
-//                 shared-memory slots into TMEM by four transposer warps as
-//                 soon as it lands (ldmatrix.trans -> tcgen05.st), and the
-//                 output MMA reads A = V^T from TMEM.  A slot is released once
-//                 the score MMA and the transposer have read it, so the ring
-//                 never waits on the softmax.  Warps: producer, score MMA,
-//                 4 softmax, 4 transposer, output MMA.
-//   ss (N = 64)   TMEM cannot hold O^T, S^T and a tile of V^T at N = 64, so
-//                 the tile stays in shared memory until the output MMA reads
-//                 V^T from it (MN-major A); the softmax writes P^T into the
-//                 dead rope slot.  Warps: producer, MMA, 4 softmax.
+// The V part of each tile is copied, transposed, from its shared-memory slots
+// into a ring of V^T blocks in TMEM by four transposer warps as soon as it
+// lands (ldmatrix.trans -> tcgen05.st), and the output MMA reads A = V^T from
+// TMEM.  A slot is released once the score MMA and the transposer have read
+// it, so the slot ring never waits on the softmax, and a V^T block is released
+// as soon as its output MMAs complete.  Warps: producer, score MMA, 4 softmax,
+// 4 transposer, output MMA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -64,10 +58,9 @@ constexpr int kTile = MLA_TILE;
 constexpr int kChunks = kDQK / 64;              // 9 column chunks per row
 constexpr uint32_t kSlotBytes = 16384;          // 128 rows x 128 B
 constexpr uint32_t kPageChunkBytes = 8192;      // 64 rows x 128 B
-constexpr int kThreadsSS = 192;                 // producer, MMA, 4 softmax warps
-constexpr int kThreadsTV = 352;                 // + 4 transposer warps, output-MMA warp
+constexpr int kThreads = 352;                   // producer, score MMA, 4 softmax, 4 transposer, output MMA
 constexpr int kMaxRing = 16;
-constexpr int kMinRing = 9;                     // a whole tile must fit: its slots are released per tile
+constexpr int kMinRing = 4;                     // the transposer may hold two chunks while the third lands
 constexpr int kMaxBatch = 4096;
 constexpr int kMaxSms = 4096;
 constexpr int kSchedHeader = 16;
@@ -75,21 +68,23 @@ constexpr int kSchedEntry = 8;
 constexpr int kSchedMagic = 0x4D4C4144;         // "MLAD"
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr uint32_t kVtCol = 256;                // tv: V^T occupies TMEM columns [256, 512)
+constexpr float kTau = 8.f;                     // log2-domain headroom before the reference max moves
+constexpr int kMaxVt = 6;                       // V^T blocks TMEM can hold beside O^T and S^T
 
 // Barrier indices inside the "misc" shared-memory region.
-constexpr int kBarFull = 0;                   // [kMaxRing]
-constexpr int kBarEmpty = kMaxRing;           // [kMaxRing]
+constexpr int kBarFull = 0;                        // [kMaxRing] slot loaded
+constexpr int kBarEmpty = kMaxRing;                // [kMaxRing] slot read by the score MMA and the transposer
 constexpr int kBarQFull = 2 * kMaxRing;
-constexpr int kBarQEmpty = 2 * kMaxRing + 1;
-constexpr int kBarSFull = 2 * kMaxRing + 2;   // [2]: one per S^T buffer
-constexpr int kBarSEmpty = 2 * kMaxRing + 4;  // [2] (tv)
-constexpr int kBarPFull = 2 * kMaxRing + 6;
-constexpr int kBarODone = 2 * kMaxRing + 7;
-constexpr int kBarVtFull = 2 * kMaxRing + 8;  // (tv)
-constexpr int kBarDrain = 2 * kMaxRing + 9;
-constexpr int kBarDrainO = 2 * kMaxRing + 10; // (tv)
-constexpr int kNumBars = 2 * kMaxRing + 11;
+constexpr int kBarQEmpty = kBarQFull + 1;
+constexpr int kBarSFull = kBarQEmpty + 1;          // [2] S^T buffer written
+constexpr int kBarSEmpty = kBarSFull + 2;          // [2] S^T buffer read into registers
+constexpr int kBarPFull = kBarSEmpty + 2;          // [2] P^T buffer written
+constexpr int kBarPEmpty = kBarPFull + 2;          // [2] output MMA of that P^T complete
+constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
+constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
+constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
+constexpr int kBarDrainO = kBarDrain + 1;
+constexpr int kNumBars = kBarDrainO + 1;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
 constexpr uint32_t kMiscRedOffset = (kNumBars * 8 + 127) / 128 * 128;
@@ -98,8 +93,9 @@ static_assert(kMiscRedOffset % 16 == 0, "reduction buffers must be 16-byte align
 template <int N>
 constexpr uint32_t misc_bytes()
 {
-    // barriers, max-reduction buffer [2][4][N], sum buffer [4][N], tmem holder, abort flag
-    return kMiscRedOffset + (2 * 4 * N + 4 * N) * 4 + 16;
+    // barriers, max-reduction buffer [4][N], sum buffer [4][N], reference max [N], shift [N],
+    // tmem holder, abort flag
+    return kMiscRedOffset + (4 * N + 4 * N + N + N) * 4 + 16;
 }
 
 struct DecodeParams {
@@ -311,54 +307,76 @@ __device__ __forceinline__ int load_pages(const int32_t *bt, int first, int npag
 }
 
 // ================================================================ decode
+// Per-shape constants.  TMEM (512 columns of 128 lanes x 32 bit) holds, left
+// to right: O^T as 4 blocks of N columns (latent dims 128j..128j+127 on the
+// lanes), NS buffers of S^T (N columns each), and a ring of NVT V^T blocks of
+// 64 columns (128 tokens as bf16 pairs; latent dims on the lanes).
 template <int N, int SQ>
 struct Cfg {
-    static constexpr bool TV = N <= 32;                    // variant (see the file header)
     static constexpr int HG = N / SQ;                      // heads per CTA
     static constexpr int NCH = N / 16;                     // 16-column TMEM chunks
+    static constexpr int NS = N <= 32 ? 2 : 1;             // S^T buffers
     static constexpr uint32_t QCHUNK = N * 128u;           // bytes: 64 columns of N rows
     static constexpr uint32_t QBYTES = kChunks * QCHUNK;   // N x 576 bf16
-    static constexpr uint32_t PBYTES = TV ? 2 * 2 * QCHUNK : 0;  // tv: 2 P^T buffers of N x 128 bf16
-    static constexpr uint32_t S_COL = 4 * N;               // S^T buffers after the 4 O^T blocks
-    static constexpr uint32_t TMEM_COLS = TV ? 512u : ((5 * N <= 256) ? 256u : 512u);
-    static constexpr int THREADS = TV ? kThreadsTV : kThreadsSS;
-    static_assert(!TV || 6 * N <= static_cast<int>(kVtCol), "O^T and S^T must fit below V^T");
+    static constexpr uint32_t PBYTES = 2 * 2 * QCHUNK;     // 2 P^T buffers of N x 128 bf16
+    static constexpr uint32_t S_COL = 4 * N;
+    static constexpr uint32_t VT_COL = (S_COL + NS * N + 63) / 64 * 64;
+    static constexpr int NVT = (512 - static_cast<int>(VT_COL)) / 64;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(NVT >= 3 && NVT <= kMaxVt, "V^T ring does not fit");
 };
 
 struct Smem {
-    uint32_t ring, q, p;     // shared-window addresses: slot ring, Q, P^T buffers (tv)
+    uint32_t ring, q, p;     // shared-window addresses: slot ring, Q, P^T buffers
     uint32_t bars;           // address of barrier 0
-    float *red, *lred;
+    float *red, *lred;       // column-max exchange [4][N], sum exchange [4][N]
+    float *mu, *shift;       // reference max [N], its last shift [N]
     uint32_t *tmem_holder;
     volatile int *abort_flag;
     __device__ __forceinline__ uint32_t bar(int i) const { return bars + 8u * i; }
     __device__ __forceinline__ uint32_t slot(int s) const { return ring + kSlotBytes * s; }
 };
 
-// Output of one range: reduce the per-row sums across the four softmax warps,
-// normalise O^T and write either the final out/lse or the fp32 piece for the
-// combine kernel.  O^T must be complete (and fenced) when this is called.
+// Output of one range: the column sums of the four softmax warps are reduced,
+// O^T is normalised and written either as the final out/lse or as the fp32
+// piece for the combine kernel.  O^T must be complete (and fenced) when this
+// is called.  `l` holds the calling thread's partial sums in the fragment
+// layout of softmax_warps.
 template <int N, int SQ>
 __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t tmem, int b, int split, int g,
-                               const float (&m)[N], float (&l)[N])
+                               const float (&l)[N / 8][2])
 {
     using C = Cfg<N, SQ>;
     constexpr int HG = C::HG;
+    constexpr int NG = N / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const int tid = threadIdx.x - 64;
+    const int c2 = 2 * (lane & 3);
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const float s = warp_sum(l[n]);
-        if (lane == 0) sm.lred[wq * N + n] = s;
-    }
+    for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            float s = l[gi][jj];
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            s += __shfl_xor_sync(0xffffffffu, s, 8);
+            s += __shfl_xor_sync(0xffffffffu, s, 16);
+            if ((lane >> 2) == 0) sm.lred[wq * N + 8 * gi + c2 + jj] = s;
+        }
     __syncwarp();
     ptx::named_bar_sync(1, 128);
+    float linv[N];
 #pragma unroll
-    for (int n = 0; n < N; ++n)
-        l[n] = (sm.lred[n] + sm.lred[N + n]) + (sm.lred[2 * N + n] + sm.lred[3 * N + n]);
+    for (int n4 = 0; n4 < N / 4; ++n4) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(sm.lred) + n4;
+        const float4 a0 = r4[0], a1 = r4[N / 4], a2 = r4[2 * (N / 4)], a3 = r4[3 * (N / 4)];
+        const float s[4] = {(a0.x + a1.x) + (a2.x + a3.x), (a0.y + a1.y) + (a2.y + a3.y),
+                            (a0.z + a1.z) + (a2.z + a3.z), (a0.w + a1.w) + (a2.w + a3.w)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) linv[4 * n4 + e] = s[e] > 0.f ? 1.f / s[e] : 0.f;
+    }
 
     const int nsplit = p.split_base[b + 1] - p.split_base[b];
     const bool final_out = nsplit <= 1;
@@ -381,7 +399,7 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
             for (int e = 0; e < 16; ++e) {
                 const int n = ch * 16 + e;
                 const int i = n / HG, hl = n % HG;
-                const float val = l[n] > 0.f ? v[e] / l[n] : 0.f;
+                const float val = v[e] * linv[n];
                 if (final_out) {
                     const int64_t o = ((static_cast<int64_t>(b) * SQ + i) * p.H + g * HG + hl) * kDV + dim;
                     p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
@@ -392,390 +410,24 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
             }
         }
     }
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        if (tid == n) {
-            const int i = n / HG, hl = n % HG;
-            const float val = l[n] > 0.f ? (m[n] + log2f(l[n])) * kLn2 : -INFINITY;
-            if (final_out)
-                p.lse[(static_cast<int64_t>(b) * SQ + i) * p.H + g * HG + hl] = val;
-            else if (write_ok)
-                p.ws_lse[(static_cast<int64_t>(piece) * SQ + i) * HG + hl] = val;
-        }
+    if (tid < N) {
+        const int n = tid;
+        const int i = n / HG, hl = n % HG;
+        const float ln = (sm.lred[n] + sm.lred[N + n]) + (sm.lred[2 * N + n] + sm.lred[3 * N + n]);
+        const float val = ln > 0.f ? (sm.mu[n] + log2f(ln)) * kLn2 : -INFINITY;
+        if (final_out)
+            p.lse[(static_cast<int64_t>(b) * SQ + i) * p.H + g * HG + hl] = val;
+        else if (write_ok)
+            p.ws_lse[(static_cast<int64_t>(piece) * SQ + i) * HG + hl] = val;
     }
     __syncwarp();
     ptx::tc_fence_before();
 }
 
-// Max over the 32 lanes of a warp for 16 columns at once: halving exchanges
-// (16 shuffles in all).  Returns, in lane l, the maximum of column l >> 1.
-__device__ __forceinline__ float warp_colmax16(float (&x)[16], int lane)
-{
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const bool hi = lane & 16;
-        const float send = hi ? x[j] : x[j + 8];
-        const float keep = hi ? x[j + 8] : x[j];
-        x[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const bool hi = lane & 8;
-        const float send = hi ? x[j] : x[j + 4];
-        const float keep = hi ? x[j + 4] : x[j];
-        x[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const bool hi = lane & 4;
-        const float send = hi ? x[j] : x[j + 2];
-        const float keep = hi ? x[j + 2] : x[j];
-        x[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-    }
-    {
-        const bool hi = lane & 2;
-        const float send = hi ? x[0] : x[1];
-        const float keep = hi ? x[1] : x[0];
-        x[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-    }
-    return fmaxf(x[0], __shfl_xor_sync(0xffffffffu, x[0], 1));
-}
-
-// ====================================================== ss variant (N = 64)
-// A tile occupies 9 consecutive ring slots starting at s0.  The four
-// (even, odd) V chunk pairs must sit in adjacent slots (an M = 128 block of
-// V^T spans both), so when the window wraps past the ring's last slot the
-// rope chunk is placed first or last to keep the wrap between two pairs.
-__device__ __forceinline__ bool rope_first_at(uint32_t s0, int R)
-{
-    if (static_cast<int>(s0) + 8 < R) return false;
-    const int w = R - 1 - static_cast<int>(s0);
-    return (w & 1) == 0;
-}
-
-__device__ __forceinline__ int pos_of_chunk(int c, bool rope_first)
-{
-    return rope_first ? (c == kChunks - 1 ? 0 : c + 1) : c;
-}
-
-// -- ss producer warp: issues every TMA load --------------------------------
+// -- producer warp: Q per range, then each tile's 9 chunks in order --------
 template <int N, int SQ>
-__device__ void ss_producer(const DecodeParams &p, const Range &w, int g, const Smem &sm,
-                             const CUtensorMap *kv_map, const CUtensorMap *q_map)
-{
-    using C = Cfg<N, SQ>;
-    const int lane = threadIdx.x & 31;
-    const int R = p.ring;
-    uint32_t cc = 0;  // chunk-slot uses so far
-    int qi = 0;       // Q loads so far
-    bool ok = true;
-    for (int b = w.b0; b <= w.b1 && ok; ++b) {
-        const int L = max(0, __ldg(p.seqlens + b));
-        const int nt = tiles_of(L);
-        const int tb = (b == w.b0) ? w.t0 : 0;
-        const int te = min((b == w.b1) ? w.t1 : nt, nt);
-        if (tb >= te) continue;
-        const int32_t *bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks;
-        const int npages = (L + kPage - 1) / kPage;
-        int win = 2 * tb;
-        int cur = load_pages(bt, win, npages, p, lane);
-        int nxt = load_pages(bt, win + 32, npages, p, lane);
-
-        if (!(ok = warp_wait(sm.bar(kBarQEmpty), (qi & 1) ^ 1, sm.abort_flag, p.err))) break;
-        ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarQFull), C::QBYTES);
-#pragma unroll 1
-        for (int i = 0; i < SQ; ++i)
-#pragma unroll 1
-            for (int c = 0; c < kChunks; ++c)
-                ptx::tma_load_2d_elect(sm.q + c * C::QCHUNK + i * C::HG * 128u, q_map, sm.bar(kBarQFull), c * 64,
-                                       (b * SQ + i) * p.H + g * C::HG);
-        ++qi;
-
-        for (int t = tb; t < te && ok; ++t) {
-            if (2 * t >= win + 32) {
-                win += 32;
-                cur = nxt;
-                nxt = load_pages(bt, win + 32, npages, p, lane);
-            }
-            const int phys0 = __shfl_sync(0xffffffffu, cur, 2 * t - win);
-            const int phys1 = __shfl_sync(0xffffffffu, cur, 2 * t + 1 - win);
-            const bool live1 = (t * kTile + kPage) < L;
-            const uint32_t bytes = live1 ? 2 * kPageChunkBytes : kPageChunkBytes;
-            const uint32_t s0 = cc % R;
-            const bool rf = rope_first_at(s0, R);
-#pragma unroll 1
-            for (int k = 0; k < kChunks; ++k) {
-                const int chunk = rf ? (k == 0 ? kChunks - 1 : k - 1) : k;
-                const uint32_t u = cc + k;
-                const int slot = static_cast<int>(u % R);
-                if (!warp_wait(sm.bar(kBarEmpty + slot), ((u / R) & 1) ^ 1, sm.abort_flag, p.err)) {
-                    ok = false;
-                    cc += k;  // uses issued so far in this tile
-                    break;
-                }
-                ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarFull + slot), bytes);
-                ptx::tma_load_3d_elect(sm.slot(slot), kv_map, sm.bar(kBarFull + slot), chunk * 64, 0, phys0);
-                if (live1)
-                    ptx::tma_load_3d_elect(sm.slot(slot) + kPageChunkBytes, kv_map, sm.bar(kBarFull + slot),
-                                           chunk * 64, 0, phys1);
-            }
-            if (ok) cc += kChunks;
-        }
-    }
-    if (!ok) {
-        // Let every load this warp issued land before the CTA exits.
-        const uint32_t first = cc > static_cast<uint32_t>(R) ? cc - R : 0;
-        for (uint32_t u = first; u < cc; ++u)
-            warp_wait(sm.bar(kBarFull + static_cast<int>(u % R)), (u / R) & 1, sm.abort_flag, p.err, false);
-    }
-}
-
-// -- ss MMA warp: issues every tcgen05.mma -----------------------------------
-template <int N, int SQ>
-__device__ void ss_mma(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
-{
-    using C = Cfg<N, SQ>;
-    constexpr uint32_t idS = ptx::idesc_bf16_f32(128, N, false, false);  // K (cache) K-major, Q K-major
-    constexpr uint32_t idO = ptx::idesc_bf16_f32(128, N, true, false);   // V^T MN-major, P^T K-major
-    const int R = p.ring;
-    uint32_t cc = 0, it = 0;
-    int qi = 0;
-    bool ok = true;
-    for (int b = w.b0; b <= w.b1 && ok; ++b) {
-        const int L = max(0, __ldg(p.seqlens + b));
-        const int nt = tiles_of(L);
-        const int tb = (b == w.b0) ? w.t0 : 0;
-        const int te = min((b == w.b1) ? w.t1 : nt, nt);
-        if (tb >= te) continue;
-        if (!(ok = warp_wait(sm.bar(kBarQFull), qi & 1, sm.abort_flag, p.err))) break;
-        ++qi;
-        ptx::tc_fence_after();
-        for (int t = tb; t < te; ++t) {
-            const uint32_t s0 = cc % R;
-            const bool rf = rope_first_at(s0, R);
-            // S^T[128 tokens x N] = K[128 x 576] . Q^T[576 x N], chunk by chunk
-#pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) {
-                const uint32_t u = cc + pos_of_chunk(c, rf);
-                const int slot = static_cast<int>(u % R);
-                if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
-                ptx::tc_fence_after();
-                const uint32_t a0 = sm.slot(slot);
-                const uint32_t b0 = sm.q + c * C::QCHUNK;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    ptx::mma_bf16_ss_elect(tmem + C::S_COL, ptx::desc_sw128(a0 + 32u * k, 16, 1024),
-                                           ptx::desc_sw128(b0 + 32u * k, 16, 1024), idS, (c | k) != 0);
-            }
-            if (!ok) break;
-            ptx::mma_commit_elect(sm.bar(kBarSFull));
-            if (t == te - 1) ptx::mma_commit_elect(sm.bar(kBarQEmpty));
-            // O^T[512 x N] += V^T[512 x 128 tokens] . P^T[128 x N]
-            if (!(ok = warp_wait(sm.bar(kBarPFull), it & 1, sm.abort_flag, p.err))) break;
-            ptx::tc_fence_after();
-            const int rope_slot = static_cast<int>((s0 + pos_of_chunk(kChunks - 1, rf)) % R);
-            const uint32_t pa = sm.slot(rope_slot);
-#pragma unroll 1
-            for (int j = 0; j < 4; ++j) {
-                const int vslot = static_cast<int>((s0 + pos_of_chunk(2 * j, rf)) % R);
-                const uint32_t va = sm.slot(vslot);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_bf16_ss_elect(tmem + j * N, ptx::desc_sw128(va + 2048u * kk, kSlotBytes, 1024),
-                                           ptx::desc_sw128(pa + (kk >> 2) * C::QCHUNK + 32u * (kk & 3), 16, 1024),
-                                           idO, (t != tb) || (kk != 0));
-                ptx::mma_commit_elect(sm.bar(kBarEmpty + vslot));
-                ptx::mma_commit_elect(sm.bar(kBarEmpty + (vslot + 1) % R));
-            }
-            ptx::mma_commit_elect(sm.bar(kBarEmpty + rope_slot));
-            ptx::mma_commit_elect(sm.bar(kBarODone));
-            cc += kChunks;
-            ++it;
-        }
-    }
-    // Every MMA this warp issued must finish before TMEM is released.
-    ptx::mma_commit_elect(sm.bar(kBarDrain));
-    warp_wait(sm.bar(kBarDrain), 0, sm.abort_flag, p.err, false);
-}
-
-// -- ss softmax / epilogue: 4 warps, thread = one TMEM lane = one token row ---
-template <int N, int SQ>
-__device__ void ss_softmax(const DecodeParams &p, const Range &w, int g, const Smem &sm, uint32_t tmem)
-{
-    using C = Cfg<N, SQ>;
-    constexpr int HG = C::HG;
-    constexpr int NCH = C::NCH;
-    constexpr bool kKeepScores = NCH <= 2;  // keep S in registers between the passes
-    const int R = p.ring;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wq = warp & 3;              // TMEM lane quadrant this warp may access
-    const int row = wq * 32 + lane;       // token row within the tile
-    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const float NEG_INF = -INFINITY;
-    uint32_t cc = 0, it = 0;
-    bool ok = true;
-
-    for (int b = w.b0; b <= w.b1 && ok; ++b) {
-        const int L = max(0, __ldg(p.seqlens + b));
-        const int nt = tiles_of(L);
-        const int tb = (b == w.b0) ? w.t0 : 0;
-        const int te = min((b == w.b1) ? w.t1 : nt, nt);
-        if (tb >= te) continue;
-        const int split = (b == w.b0) ? w.split0 : 0;
-        const int nvis0 = max(0, L - SQ + 1);  // tokens visible to query position 0
-        float m[N], l[N];
-#pragma unroll
-        for (int n = 0; n < N; ++n) { m[n] = NEG_INF; l[n] = 0.f; }
-
-        for (int t = tb; t < te; ++t) {
-            const uint32_t s0 = cc % R;
-            const bool rf = rope_first_at(s0, R);
-            const bool got_s = wait_bounded(sm.bar(kBarSFull), it & 1, sm.abort_flag, p.err);
-            __syncwarp();
-            ok = ptx::named_bar_and(1, 128, got_s);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            const int tok = t * kTile + row;
-            const bool vis0 = tok < nvis0, vis1 = tok < L;
-            float *red = sm.red + (it & 1) * 4 * N;
-            // pass 1: masked log2-domain scores and their per-column maximum
-            float sc[kKeepScores ? NCH : 1][16];
-#pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                float v[16];
-                ptx::tmem_ld16(tmem + lane_base + C::S_COL + ch * 16, v);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = ch * 16 + e;
-                    const bool vis = (SQ == 2 && n >= HG) ? vis1 : vis0;
-                    v[e] = vis ? v[e] * p.scale_log2 : NEG_INF;
-                    if (kKeepScores) sc[kKeepScores ? ch : 0][e] = v[e];
-                }
-                const float cmax = warp_colmax16(v, lane);
-                if ((lane & 1) == 0) red[wq * N + ch * 16 + (lane >> 1)] = cmax;
-            }
-            __syncwarp();
-            ptx::named_bar_sync(1, 128);
-            // pass 2: running max, weights, P^T into the rope slot, running sums
-            const int rope_slot = static_cast<int>((s0 + pos_of_chunk(kChunks - 1, rf)) % R);
-            const uint32_t pa = sm.slot(rope_slot) + (row >> 6) * C::QCHUNK;
-            const uint32_t pcol = static_cast<uint32_t>(row & 63);
-            bool any_rescale = false;
-            float alpha[N];
-#pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                float v[16];
-                if (kKeepScores) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = sc[kKeepScores ? ch : 0][e];
-                } else {
-                    ptx::tmem_ld16(tmem + lane_base + C::S_COL + ch * 16, v);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int n = ch * 16 + e;
-                        const bool vis = (SQ == 2 && n >= HG) ? vis1 : vis0;
-                        v[e] = vis ? v[e] * p.scale_log2 : NEG_INF;
-                    }
-                }
-                float tmax[16];
-                {
-                    const float4 *r4 = reinterpret_cast<const float4 *>(red + ch * 16);
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 a0 = r4[e4], a1 = r4[N / 4 + e4], a2 = r4[2 * (N / 4) + e4],
-                                     a3 = r4[3 * (N / 4) + e4];
-                        tmax[4 * e4 + 0] = fmaxf(fmaxf(a0.x, a1.x), fmaxf(a2.x, a3.x));
-                        tmax[4 * e4 + 1] = fmaxf(fmaxf(a0.y, a1.y), fmaxf(a2.y, a3.y));
-                        tmax[4 * e4 + 2] = fmaxf(fmaxf(a0.z, a1.z), fmaxf(a2.z, a3.z));
-                        tmax[4 * e4 + 3] = fmaxf(fmaxf(a0.w, a1.w), fmaxf(a2.w, a3.w));
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = ch * 16 + e;
-                    const float mnew = fmaxf(m[n], tmax[e]);
-                    // The reference max follows the true running max, so the
-                    // largest weight of a range is exactly 1.
-                    const bool need = mnew > m[n];
-                    alpha[n] = need ? ptx::ex2_approx(m[n] - mnew) : 1.f;
-                    if (need) {
-                        m[n] = mnew;
-                        any_rescale = true;
-                    }
-                    const float mu = (m[n] == NEG_INF) ? 0.f : m[n];
-                    const float pr = ptx::ex2_approx(v[e] - mu);  // masked entries: 2^-inf = 0
-                    l[n] = l[n] * alpha[n] + pr;
-                    const uint32_t addr = pa + n * 128u + ((((pcol >> 3) ^ static_cast<uint32_t>(n & 7)) << 4)) +
-                                          ((pcol & 7u) << 1);
-                    ptx::st_shared_b16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(pr)));
-                }
-            }
-            // rows past the end of the sequence: make their V bytes zero so
-            // that P = 0 meets finite values in the output MMA
-            if (tok >= L) {
-#pragma unroll 1
-                for (int c = 0; c < kChunks - 1; ++c) {
-                    const int vs = static_cast<int>((s0 + pos_of_chunk(c, rf)) % R);
-                    const uint32_t ra = sm.slot(vs) + row * 128u;
-#pragma unroll
-                    for (int q16 = 0; q16 < 8; ++q16) ptx::st_shared_zero16(ra + q16 * 16u);
-                }
-            }
-            __syncwarp();
-            // rescale the O^T columns whose reference max moved (not needed
-            // on the first tile of a range: its output MMA overwrites O^T)
-            if (any_rescale && t != tb) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                    for (int ch = 0; ch < NCH; ++ch) {
-                        float v[16];
-                        const uint32_t ta = tmem + lane_base + j * N + ch * 16;
-                        ptx::tmem_ld16(ta, v);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] *= alpha[ch * 16 + e];
-                        ptx::tmem_st16(ta, v);
-                    }
-                }
-                ptx::tmem_wait_st();
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(sm.bar(kBarPFull));
-            cc += kChunks;
-            ++it;
-        }
-        if (!ok) break;
-
-        // ---- epilogue of this range
-        const bool got_o = wait_bounded(sm.bar(kBarODone), (it - 1) & 1, sm.abort_flag, p.err);
-        __syncwarp();
-        ok = ptx::named_bar_and(1, 128, got_o);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        range_epilogue<N, SQ>(p, sm, tmem, b, split, g, m, l);
-    }
-}
-
-// ====================================================== tv variant (N <= 32)
-// K position, in the output MMA, of token r of a tile.  ldmatrix.trans hands
-// each thread token pairs (2q, 2q+1) and (8+2q, 9+2q) of a 16-token group for
-// one latent dim; stored as TMEM columns 2q and 2q+1 of that dim's lane they
-// give the order 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15 within each group.
-// P^T is written in the same order, so the contraction is unchanged.
-__device__ __forceinline__ int tv_kpos(int r)
-{
-    const int g = r & ~15, rr = r & 15;
-    return g + (rr < 8 ? 2 * (rr & ~1) + (rr & 1) : 2 * ((rr - 8) & ~1) + 2 + (rr & 1));
-}
-
-// -- tv producer warp: Q per range, then each tile's 9 chunks in order ----
-template <int N, int SQ>
-__device__ void tv_producer(const DecodeParams &p, const Range &w, int g, const Smem &sm,
-                            const CUtensorMap *kv_map, const CUtensorMap *q_map)
+__device__ void producer_warp(const DecodeParams &p, const Range &w, int g, const Smem &sm,
+                              const CUtensorMap *kv_map, const CUtensorMap *q_map)
 {
     using C = Cfg<N, SQ>;
     const int lane = threadIdx.x & 31;
@@ -841,9 +493,9 @@ __device__ void tv_producer(const DecodeParams &p, const Range &w, int g, const 
     }
 }
 
-// -- tv score-MMA warp: S^T(t) into S buffer t & 1, chunk by chunk --------
+// -- score-MMA warp: S^T(t) into S buffer t % NS, chunk by chunk ------------
 template <int N, int SQ>
-__device__ void tv_s_mma(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
+__device__ void score_mma_warp(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
     constexpr uint32_t idS = ptx::idesc_bf16_f32(128, N, false, false);  // K (cache) K-major, Q K-major
@@ -861,12 +513,11 @@ __device__ void tv_s_mma(const DecodeParams &p, const Range &w, const Smem &sm, 
         ++qi;
         ptx::tc_fence_after();
         for (int t = tb; t < te && ok; ++t) {
-            // the softmax has finished reading S^T(it - 2) from this buffer
-            if (it >= 2 &&
-                !(ok = warp_wait(sm.bar(kBarSEmpty + (it & 1)), ((it >> 1) & 1) ^ 1, sm.abort_flag, p.err)))
-                break;
+            const uint32_t sb = it % C::NS, su = it / C::NS;
+            // the softmax has read the previous S^T of this buffer into registers
+            if (su >= 1 && !(ok = warp_wait(sm.bar(kBarSEmpty + sb), (su & 1) ^ 1, sm.abort_flag, p.err))) break;
             ptx::tc_fence_after();
-            const uint32_t d = tmem + C::S_COL + (it & 1) * N;
+            const uint32_t d = tmem + C::S_COL + sb * N;
 #pragma unroll 1
             for (int c = 0; c < kChunks; ++c) {
                 const uint32_t u = cc + c;
@@ -889,7 +540,7 @@ __device__ void tv_s_mma(const DecodeParams &p, const Range &w, const Smem &sm, 
                 }
             }
             if (!ok) break;
-            ptx::mma_commit_elect(sm.bar(kBarSFull + (it & 1)));
+            ptx::mma_commit_elect(sm.bar(kBarSFull + sb));
             if (t == te - 1) ptx::mma_commit_elect(sm.bar(kBarQEmpty));
             cc += kChunks;
             ++it;
@@ -899,33 +550,42 @@ __device__ void tv_s_mma(const DecodeParams &p, const Range &w, const Smem &sm, 
     warp_wait(sm.bar(kBarDrain), 0, sm.abort_flag, p.err, false);
 }
 
-// -- tv output-MMA warp: O^T += V^T (TMEM) . P^T (shared memory) ----------
+// -- output-MMA warp: O^T += V^T (TMEM ring) . P^T (shared memory) ----------
+// Tile t's four 128-dim blocks are V^T blocks v = 4t .. 4t+3 of the ring; each
+// block is handed back to the transposer as soon as its 8 MMAs complete.
 template <int N, int SQ>
-__device__ void tv_o_mma(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
+__device__ void output_mma_warp(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
     constexpr uint32_t idO = ptx::idesc_bf16_f32(128, N, false, false);  // A in TMEM, P^T K-major
-    uint32_t it = 0;
+    constexpr uint32_t NVT = C::NVT;
+    uint32_t it = 0, v = 0;
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
         const int L = max(0, __ldg(p.seqlens + b));
         const int nt = tiles_of(L);
         const int tb = (b == w.b0) ? w.t0 : 0;
         const int te = min((b == w.b1) ? w.t1 : nt, nt);
-        for (int t = tb; t < te; ++t) {
-            if (!(ok = warp_wait(sm.bar(kBarPFull), it & 1, sm.abort_flag, p.err))) break;
-            if (!(ok = warp_wait(sm.bar(kBarVtFull), it & 1, sm.abort_flag, p.err))) break;
+        for (int t = tb; t < te && ok; ++t) {
+            const uint32_t pb = it & 1, pu = it >> 1;
+            if (!(ok = warp_wait(sm.bar(kBarPFull + pb), pu & 1, sm.abort_flag, p.err))) break;
             ptx::tc_fence_after();
-            const uint32_t pa = sm.p + (it & 1) * 2 * C::QCHUNK;
+            const uint32_t pa = sm.p + pb * 2 * C::QCHUNK;
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) {
+                const uint32_t vb = v % NVT, vu = v / NVT;
+                if (!(ok = warp_wait(sm.bar(kBarVtFull + vb), vu & 1, sm.abort_flag, p.err))) break;
+                ptx::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_bf16_ts_elect(tmem + j * N, tmem + kVtCol + 64 * j + 8 * kk,
+                    ptx::mma_bf16_ts_elect(tmem + j * N, tmem + C::VT_COL + 64 * vb + 8 * kk,
                                            ptx::desc_sw128(pa + (kk >> 2) * C::QCHUNK + 32u * (kk & 3), 16, 1024),
                                            idO, (t != tb) || (kk != 0));
+                ptx::mma_commit_elect(sm.bar(kBarVtEmpty + vb));
+                ++v;
             }
-            ptx::mma_commit_elect(sm.bar(kBarODone));
+            if (!ok) break;
+            ptx::mma_commit_elect(sm.bar(kBarPEmpty + pb));
             ++it;
         }
     }
@@ -933,43 +593,39 @@ __device__ void tv_o_mma(const DecodeParams &p, const Range &w, const Smem &sm, 
     warp_wait(sm.bar(kBarDrainO), 0, sm.abort_flag, p.err, false);
 }
 
-// -- tv transposer: 4 warps copy V(t) into TMEM as V^T --------------------
+// -- transposer: 4 warps copy V(t) into the TMEM ring as V^T ----------------
 // Warp q owns TMEM lanes 32q..32q+31, i.e. latent dims 128j + 32q + (0..31)
 // of every 128-dim block j: half of chunk 2j + q/2.  Per 16 dims x 16 tokens
 // one ldmatrix.x4.trans feeds one tcgen05.st.16x256b.
 template <int N, int SQ>
-__device__ void tv_transposer(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
+__device__ void transposer_warps(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
+    using C = Cfg<N, SQ>;
+    constexpr uint32_t NVT = C::NVT;
     const uint32_t R = static_cast<uint32_t>(p.ring);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;
-    const int ttid = threadIdx.x - 192;  // 0..127 within the transposer group
-    uint32_t cc = 0, it = 0, od = 0;
+    uint32_t cc = 0, v = 0;
     bool ok = true;
-    // ldmatrix row addresses: lane -> (matrix mi, row rr)
+    // ldmatrix row addresses: lane -> (matrix mi, row rr).  Matrices 0 and 2
+    // take tokens {0,1,4,5,8,9,12,13} of a 16-token group, matrices 1 and 3
+    // tokens {2,3,6,7,10,11,14,15}: thread t then receives token pairs
+    // (4(t%4), 4(t%4)+1) and (4(t%4)+2, 4(t%4)+3), which the 16x256b store puts
+    // in TMEM columns 2(t%4) and 2(t%4)+1 -- tokens in natural order.
     const int mi = lane >> 3, rr = lane & 7;
-    const int tok_in = rr + 8 * (mi & 1);        // token within a 16-token group
-    const int dim_in = 8 * (mi >> 1);            // dim offset within a 16-dim half
+    const int tok_in = 4 * (rr >> 1) + (rr & 1) + 2 * (mi & 1);  // token within a 16-token group
+    const int dim_in = 8 * (mi >> 1);                             // dim offset within a 16-dim half
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
         const int L = max(0, __ldg(p.seqlens + b));
         const int nt = tiles_of(L);
         const int tb = (b == w.b0) ? w.t0 : 0;
         const int te = min((b == w.b1) ? w.t1 : nt, nt);
         for (int t = tb; t < te; ++t) {
-            // V^T buffer free: the output MMA of the previous tile is complete
-            bool good = true;
-            while (od < it) {
-                good = good && wait_bounded(sm.bar(kBarODone), od & 1, sm.abort_flag, p.err);
-                ++od;
-            }
-            __syncwarp();
-            if (!(ok = ptx::named_bar_and(2, 128, good))) break;
-            ptx::tc_fence_after();
             const int valid = L - t * kTile;  // tokens of this tile inside the sequence
-            // Warp q's share of chunk j (latent block j): 16 ldmatrix.x4 =
-            // 64 registers.  All 16 loads of a chunk are in flight together,
-            // and the next chunk's loads are issued before this chunk is
-            // stored, so the shared-memory latency is paid about once per chunk.
+            // Warp q's share of block j: 16 ldmatrix.x4 = 64 registers.  All
+            // 16 loads of a block are in flight together, and the next
+            // block's loads are issued before this block is stored, so the
+            // shared-memory latency is paid about once per block.
             auto wait_chunk = [&](int j, uint32_t &slot_out) -> bool {
                 const uint32_t u = cc + 2 * j + (q >> 1);
                 slot_out = u % R;
@@ -989,7 +645,7 @@ __device__ void tv_transposer(const DecodeParams &p, const Range &w, const Smem 
                     }
                 }
             };
-            auto store_chunk = [&](int j, uint32_t (&r)[64]) {
+            auto store_chunk = [&](uint32_t vb, uint32_t (&r)[64]) {
                 if (valid < kTile) {
                     // tokens past the sequence end: their P is zero, make V^T zero too
 #pragma unroll
@@ -998,7 +654,7 @@ __device__ void tv_transposer(const DecodeParams &p, const Range &w, const Smem 
                         for (int gi = 0; gi < 8; ++gi)
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                const int t0 = 16 * gi + 8 * (i & 1) + 2 * (lane & 3);
+                                const int t0 = 16 * gi + 4 * (lane & 3) + 2 * (i & 1);
                                 uint32_t &x = r[32 * h + 4 * gi + i];
                                 if (t0 >= valid) x = 0;
                                 else if (t0 + 1 >= valid) x &= 0xFFFFu;
@@ -1008,11 +664,11 @@ __device__ void tv_transposer(const DecodeParams &p, const Range &w, const Smem 
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int gg = 0; gg < 2; ++gg) {
-                        uint32_t v[16];
+                        uint32_t x[16];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) v[k] = r[32 * h + 16 * gg + k];
+                        for (int k = 0; k < 16; ++k) x[k] = r[32 * h + 16 * gg + k];
                         ptx::tmem_st_16x256b_x4(
-                            tmem + (static_cast<uint32_t>(32 * q + 16 * h) << 16) + kVtCol + 64 * j + 32 * gg, v);
+                            tmem + (static_cast<uint32_t>(32 * q + 16 * h) << 16) + C::VT_COL + 64 * vb + 32 * gg, x);
                     }
             };
             uint32_t ra[64], rb[64];
@@ -1029,50 +685,60 @@ __device__ void tv_transposer(const DecodeParams &p, const Range &w, const Smem 
                     if (!(ok = wait_chunk(j + 1, slot_nxt))) break;
                     load_chunk(slot_nxt, nxt);
                 }
-                store_chunk(j, cur);
-                // the stores consumed this chunk's loaded registers: release
-                // this warp's share of the slot
+                // ring block free: the output MMA that read it last is complete
+                const uint32_t vb = v % NVT, vu = v / NVT;
+                if (vu >= 1 && !(ok = warp_wait(sm.bar(kBarVtEmpty + vb), (vu & 1) ^ 1, sm.abort_flag, p.err)))
+                    break;
+                ptx::tc_fence_after();
+                store_chunk(vb, cur);
+                // the stores consumed this block's registers: release this
+                // warp's share of the slot
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(sm.bar(kBarEmpty + static_cast<int>(slot_cur)));
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(sm.bar(kBarVtFull + vb));
+                ++v;
             }
             if (!ok) break;
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            __syncwarp();
-            ptx::named_bar_sync(2, 128);
-            if (ttid == 0) ptx::mbar_arrive(sm.bar(kBarVtFull));
             cc += kChunks;
-            ++it;
         }
     }
 }
 
-// -- tv softmax / epilogue: 4 warps, thread = one TMEM lane = one token row
+// -- softmax / epilogue: 4 warps over the 128 token rows of S^T --------------
+// S^T is read in the tensor-core fragment layout (tcgen05.ld 16x256b): in
+// each 16-row half hf of its warp's 32 rows, thread t holds rows t/4 and
+// t/4 + 8 for the two columns 2(t%4), 2(t%4)+1 of every 8-column group, so a
+// thread owns N/4 columns and 4 token rows.  P^T goes to shared memory with
+// stmatrix.trans straight from that layout (8 tokens x 2 bytes per row).
+//
+// Scores are kept in the log2 domain relative to a per-column reference max
+// mu.  A tile only moves mu -- with an exact column max over the tile, a
+// rescale of the running sums and of O^T -- when some score exceeds mu by more
+// than 2^kTau (and always on the first tile of a range); otherwise its
+// weights 2^(s - mu) are at most 2^kTau and nothing is rescaled.  Every weight
+// of a column is taken relative to the same mu as its sum, so the result is
+// the same softmax.
 template <int N, int SQ>
-__device__ void tv_softmax(const DecodeParams &p, const Range &w, int g, const Smem &sm, uint32_t tmem)
+__device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
     constexpr int HG = C::HG;
     constexpr int NCH = C::NCH;
+    constexpr int NG = N / 8;             // 8-column groups
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wq = warp & 3;              // TMEM lane quadrant this warp may access
-    const int row = wq * 32 + lane;       // token row within the tile
+    const int stid = threadIdx.x - 64;    // 0..127 within the softmax group
+    const int c2 = 2 * (lane & 3);        // this thread's first column in each group
+    const int r8 = lane >> 2;             // its token row within an 8-row block
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const int kp = tv_kpos(row);          // this row's K position in the output MMA
+    // stmatrix: lanes 8i..8i+7 address matrix i = (token block i & 1, group offset i >> 1)
+    const int st_blk = (lane >> 3) & 1, st_go = lane >> 4, st_row = lane & 7;
     const float NEG_INF = -INFINITY;
     uint32_t it = 0;   // tiles processed
-    uint32_t od = 0;   // output-MMA completions observed
     bool ok = true;
-    // Observe the output MMAs in order up to (not including) tile `upto`.
-    auto observe_o = [&](uint32_t upto) -> bool {
-        bool good = true;
-        while (od < upto) {
-            good = good && wait_bounded(sm.bar(kBarODone), od & 1, sm.abort_flag, p.err);
-            ++od;
-        }
-        __syncwarp();
-        return ptx::named_bar_and(1, 128, good);
-    };
 
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
         const int L = max(0, __ldg(p.seqlens + b));
@@ -1082,122 +748,176 @@ __device__ void tv_softmax(const DecodeParams &p, const Range &w, int g, const S
         if (tb >= te) continue;
         const int split = (b == w.b0) ? w.split0 : 0;
         const int nvis0 = max(0, L - SQ + 1);  // tokens visible to query position 0
-        float m[N], l[N];
+        float l[NG][2], mu[NG][2];             // this thread's columns: running sums, reference max
 #pragma unroll
-        for (int n = 0; n < N; ++n) { m[n] = NEG_INF; l[n] = 0.f; }
+        for (int gi = 0; gi < NG; ++gi) l[gi][0] = l[gi][1] = mu[gi][0] = mu[gi][1] = 0.f;
+        bool wait_ok = true;  // a failed wait is carried to the next agreement point
 
         for (int t = tb; t < te; ++t) {
-            const bool got_s = wait_bounded(sm.bar(kBarSFull + (it & 1)), (it >> 1) & 1, sm.abort_flag, p.err);
-            __syncwarp();
-            ok = ptx::named_bar_and(1, 128, got_s);
-            if (!ok) break;
+            const uint32_t sb = it % C::NS, su = it / C::NS;
+            wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
             ptx::tc_fence_after();
-            const uint32_t s_taddr = tmem + lane_base + C::S_COL + (it & 1) * N;
-            const int tok = t * kTile + row;
-            const bool vis0 = tok < nvis0, vis1 = tok < L;
-            float *red = sm.red + (it & 1) * 4 * N;
-            // pass 1: masked log2-domain scores and their per-column maximum
-            float sc[NCH][16];
+            uint32_t raw[2][4 * NG];
 #pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                ptx::tmem_ld16(s_taddr + ch * 16, sc[ch]);
-                ptx::tmem_wait_ld();
-            }
+            for (int hf = 0; hf < 2; ++hf)
+                ptx::tmem_ld_16x256b(tmem + (static_cast<uint32_t>(32 * wq + 16 * hf) << 16) + C::S_COL + sb * N,
+                                     raw[hf]);
+            ptx::tmem_wait_ld();
             // S^T(it) is in registers: its TMEM buffer may be overwritten
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(sm.bar(kBarSEmpty + (it & 1)));
+            if (lane == 0) ptx::mbar_arrive(sm.bar(kBarSEmpty + sb));
+
+            // pass 1: masked log2-domain scores relative to mu
+            const bool first = (t == tb);
+            const int tok0 = t * kTile + 32 * wq + r8;
+            float d[2][NG][4];
+            bool flag = first || !wait_ok;
 #pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                float v[16];
+            for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = ch * 16 + e;
-                    const bool vis = (SQ == 2 && n >= HG) ? vis1 : vis0;
-                    sc[ch][e] = vis ? sc[ch][e] * p.scale_log2 : NEG_INF;
-                    v[e] = sc[ch][e];
-                }
-                const float cmax = warp_colmax16(v, lane);
-                if ((lane & 1) == 0) red[wq * N + ch * 16 + (lane >> 1)] = cmax;
-            }
+                for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int tok = tok0 + 16 * hf + 8 * (j >> 1);
+                        const int n = 8 * gi + c2 + (j & 1);
+                        const bool vis = (SQ == 2 && n >= HG) ? (tok < L) : (tok < nvis0);
+                        const float s = __uint_as_float(raw[hf][4 * gi + j]);
+                        d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, -mu[gi][j & 1]) : NEG_INF;
+                        flag = flag || (d[hf][gi][j] > kTau);
+                    }
             __syncwarp();
-            ptx::named_bar_sync(1, 128);
-            // pass 2: running max, weights, P^T (permuted K order), running sums
-            const uint32_t pa = sm.p + (it & 1) * 2 * C::QCHUNK + (kp >> 6) * C::QCHUNK;
-            const uint32_t pcol = static_cast<uint32_t>(kp & 63);
-            bool any_rescale = false;
-            float alpha[N];
+            if (ptx::named_bar_or(1, 128, flag)) {
+                if (!(ok = ptx::named_bar_and(1, 128, wait_ok))) break;
+                // exact column max of this tile (relative to mu): over the
+                // thread's 4 rows, the 8 lanes sharing its columns, the 4 warps
+                float cm[NG][2];
 #pragma unroll
-            for (int ch = 0; ch < NCH; ++ch) {
-                float tmax[16];
-                {
-                    const float4 *r4 = reinterpret_cast<const float4 *>(red + ch * 16);
+                for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 a0 = r4[e4], a1 = r4[N / 4 + e4], a2 = r4[2 * (N / 4) + e4],
-                                     a3 = r4[3 * (N / 4) + e4];
-                        tmax[4 * e4 + 0] = fmaxf(fmaxf(a0.x, a1.x), fmaxf(a2.x, a3.x));
-                        tmax[4 * e4 + 1] = fmaxf(fmaxf(a0.y, a1.y), fmaxf(a2.y, a3.y));
-                        tmax[4 * e4 + 2] = fmaxf(fmaxf(a0.z, a1.z), fmaxf(a2.z, a3.z));
-                        tmax[4 * e4 + 3] = fmaxf(fmaxf(a0.w, a1.w), fmaxf(a2.w, a3.w));
+                    for (int jj = 0; jj < 2; ++jj) {
+                        float m = fmaxf(fmaxf(d[0][gi][jj], d[0][gi][jj + 2]), fmaxf(d[1][gi][jj], d[1][gi][jj + 2]));
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                        cm[gi][jj] = m;
+                    }
+                if (r8 == 0) {
+#pragma unroll
+                    for (int gi = 0; gi < NG; ++gi)
+                        *reinterpret_cast<float2 *>(sm.red + wq * N + 8 * gi + c2) = make_float2(cm[gi][0], cm[gi][1]);
+                }
+                __syncwarp();
+                ptx::named_bar_sync(1, 128);
+                // shift of column n: on the first tile the exact max (none if
+                // the column saw no token), afterwards only upwards
+                if (stid < N) {
+                    const int n = stid;
+                    const float x = fmaxf(fmaxf(sm.red[n], sm.red[N + n]), fmaxf(sm.red[2 * N + n], sm.red[3 * N + n]));
+                    const float sh = first ? (x == NEG_INF ? 0.f : x) : fmaxf(x, 0.f);
+                    sm.shift[n] = sh;
+                    sm.mu[n] = (first ? 0.f : sm.mu[n]) + sh;
+                }
+                __syncwarp();
+                ptx::named_bar_sync(1, 128);
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) {
+                    const float2 s2 = *reinterpret_cast<const float2 *>(sm.shift + 8 * gi + c2);
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const float sh = jj ? s2.y : s2.x;
+                        mu[gi][jj] += sh;
+                        if (!first) l[gi][jj] *= ptx::ex2_approx(-sh);
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            d[hf][gi][jj] -= sh;
+                            d[hf][gi][jj + 2] -= sh;
+                        }
                     }
                 }
+                if (!first) {
+                    // O^T is rescaled once the previous tile's output MMA is complete
+                    const uint32_t pp = it - 1;
+                    wait_ok = wait_bounded(sm.bar(kBarPEmpty + (pp & 1)), (pp >> 1) & 1, sm.abort_flag, p.err) &&
+                              wait_ok;
+                    ptx::tc_fence_after();
+#pragma unroll 1
+                    for (int ch = 0; ch < NCH; ++ch) {
+                        float a[16];
+                        const float4 *s4 = reinterpret_cast<const float4 *>(sm.shift + 16 * ch);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = ch * 16 + e;
-                    const float mnew = fmaxf(m[n], tmax[e]);
-                    // The reference max follows the true running max, so the
-                    // largest weight of a range is exactly 1.
-                    const bool need = mnew > m[n];
-                    alpha[n] = need ? ptx::ex2_approx(m[n] - mnew) : 1.f;
-                    if (need) {
-                        m[n] = mnew;
-                        any_rescale = true;
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 v4 = s4[e4];
+                            a[4 * e4 + 0] = ptx::ex2_approx(-v4.x);
+                            a[4 * e4 + 1] = ptx::ex2_approx(-v4.y);
+                            a[4 * e4 + 2] = ptx::ex2_approx(-v4.z);
+                            a[4 * e4 + 3] = ptx::ex2_approx(-v4.w);
+                        }
+#pragma unroll 1
+                        for (int j = 0; j < 4; ++j) {
+                            float x[16];
+                            const uint32_t ta = tmem + lane_base + j * N + ch * 16;
+                            ptx::tmem_ld16(ta, x);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) x[e] *= a[e];
+                            ptx::tmem_st16(ta, x);
+                        }
                     }
-                    const float mu = (m[n] == NEG_INF) ? 0.f : m[n];
-                    const float pr = ptx::ex2_approx(sc[ch][e] - mu);  // masked entries: 2^-inf = 0
-                    l[n] = l[n] * alpha[n] + pr;
-                    const uint32_t addr = pa + n * 128u + ((((pcol >> 3) ^ static_cast<uint32_t>(n & 7)) << 4)) +
-                                          ((pcol & 7u) << 1);
-                    ptx::st_shared_b16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(pr)));
+                    ptx::tmem_wait_st();
                 }
             }
-            // The previous tile's output MMA must be complete before O^T is
-            // rescaled (observed every tile, so the wait never lags).
-            if (!(ok = observe_o(it))) break;
-            ptx::tc_fence_after();
-            if (any_rescale && t != tb) {
+
+            // pass 2: weights -> P^T and the running sums, into P buffer it & 1
+            // once the output MMA of tile it - 2 is done
+            if (it >= 2)
+                wait_ok = wait_bounded(sm.bar(kBarPEmpty + (it & 1)), ((it >> 1) & 1) ^ 1, sm.abort_flag, p.err) &&
+                          wait_ok;
+            const uint32_t pbuf = sm.p + (it & 1) * 2 * C::QCHUNK;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[NG][2];
 #pragma unroll
-                    for (int ch = 0; ch < NCH; ++ch) {
-                        float v[16];
-                        const uint32_t ta = tmem + lane_base + j * N + ch * 16;
-                        ptx::tmem_ld16(ta, v);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] *= alpha[ch * 16 + e];
-                        ptx::tmem_st16(ta, v);
-                    }
+                for (int gi = 0; gi < NG; ++gi) {
+                    const float p0 = ptx::ex2_approx(d[hf][gi][0]);  // masked entries: 2^-inf = 0
+                    const float p1 = ptx::ex2_approx(d[hf][gi][1]);
+                    const float p2 = ptx::ex2_approx(d[hf][gi][2]);
+                    const float p3 = ptx::ex2_approx(d[hf][gi][3]);
+                    l[gi][0] += p0 + p2;
+                    l[gi][1] += p1 + p3;
+                    pk[gi][0] = ptx::pack_bf16x2(p0, p1);  // token row r8
+                    pk[gi][1] = ptx::pack_bf16x2(p2, p3);  // token row r8 + 8
                 }
-                ptx::tmem_wait_st();
+                // P^T rows n, K positions = tokens of the tile (natural order)
+                const int kb = 32 * wq + 16 * hf + 8 * st_blk;  // first token of this lane's matrix
+                const uint32_t kbase = pbuf + (kb >> 6) * C::QCHUNK;
+                const uint32_t kchunk = static_cast<uint32_t>((kb & 63) >> 3);
+#pragma unroll
+                for (int gp = 0; gp < NG / 2; ++gp) {
+                    const int n = 8 * (2 * gp + st_go) + st_row;
+                    const uint32_t addr = kbase + n * 128u + ((kchunk ^ static_cast<uint32_t>(n & 7)) << 4);
+                    ptx::stsm_x4_trans(addr, pk[2 * gp][0], pk[2 * gp][1], pk[2 * gp + 1][0], pk[2 * gp + 1][1]);
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(sm.bar(kBarPFull));
+            ptx::mbar_arrive(sm.bar(kBarPFull + (it & 1)));
             ++it;
         }
         if (!ok) break;
-        if (!(ok = observe_o(it))) break;
+        // ---- epilogue of this range: its last output MMA must be complete
+        const uint32_t pp = it - 1;
+        wait_ok = wait_bounded(sm.bar(kBarPEmpty + (pp & 1)), (pp >> 1) & 1, sm.abort_flag, p.err) && wait_ok;
+        __syncwarp();
+        if (!(ok = ptx::named_bar_and(1, 128, wait_ok))) break;
         ptx::tc_fence_after();
-        range_epilogue<N, SQ>(p, sm, tmem, b, split, g, m, l);
+        range_epilogue<N, SQ>(p, sm, tmem, b, split, g, l);
     }
 }
 
-// ============================================================== kernels
-// Shared prologue of both variants: schedule check, shared-memory carve-up,
-// barrier initialisation and TMEM allocation.  Returns false (uniformly) when
-// this CTA has no work.
+// ============================================================== kernel
+// Prologue: schedule check, shared-memory carve-up, barrier initialisation
+// and TMEM allocation.  Returns false (uniformly) when this CTA has no work.
 template <int N, int SQ>
 __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtensorMap *kv_map,
                                              const CUtensorMap *q_map, uint8_t *smem_raw, Smem &sm, Range &w,
@@ -1224,25 +944,30 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     uint8_t *misc = gbase + p.ring * kSlotBytes + C::QBYTES + C::PBYTES;
     sm.bars = ptx::smem_addr(misc);
     sm.red = reinterpret_cast<float *>(misc + kMiscRedOffset);
-    sm.lred = sm.red + 2 * 4 * N;
-    sm.tmem_holder = reinterpret_cast<uint32_t *>(sm.lred + 4 * N);
+    sm.lred = sm.red + 4 * N;
+    sm.mu = sm.lred + 4 * N;
+    sm.shift = sm.mu + N;
+    sm.tmem_holder = reinterpret_cast<uint32_t *>(sm.shift + N);
     sm.abort_flag = reinterpret_cast<volatile int *>(sm.tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ring; ++s) {
             ptx::mbar_init(sm.bar(kBarFull + s), 1);
-            ptx::mbar_init(sm.bar(kBarEmpty + s), C::TV ? 3 : 1);
+            ptx::mbar_init(sm.bar(kBarEmpty + s), 3);
         }
         ptx::mbar_init(sm.bar(kBarQFull), 1);
         ptx::mbar_init(sm.bar(kBarQEmpty), 1);
-        ptx::mbar_init(sm.bar(kBarSFull), 1);
-        ptx::mbar_init(sm.bar(kBarSFull + 1), 1);
-        ptx::mbar_init(sm.bar(kBarSEmpty), 4);
-        ptx::mbar_init(sm.bar(kBarSEmpty + 1), 4);
-        ptx::mbar_init(sm.bar(kBarPFull), 128);
-        ptx::mbar_init(sm.bar(kBarODone), 1);
-        ptx::mbar_init(sm.bar(kBarVtFull), 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(sm.bar(kBarSFull + i), 1);
+            ptx::mbar_init(sm.bar(kBarSEmpty + i), 4);
+            ptx::mbar_init(sm.bar(kBarPFull + i), 128);
+            ptx::mbar_init(sm.bar(kBarPEmpty + i), 1);
+        }
+        for (int i = 0; i < kMaxVt; ++i) {
+            ptx::mbar_init(sm.bar(kBarVtFull + i), 4);
+            ptx::mbar_init(sm.bar(kBarVtEmpty + i), 1);
+        }
         ptx::mbar_init(sm.bar(kBarDrain), 1);
         ptx::mbar_init(sm.bar(kBarDrainO), 1);
         *sm.abort_flag = 0;
@@ -1274,10 +999,12 @@ __device__ __forceinline__ void decode_teardown(uint32_t tmem)
     }
 }
 
+// Warps: 0 producer, 1 score MMA (and TMEM owner), 2-5 softmax + epilogue,
+// 6-9 transposer, 10 output MMA.
 template <int N, int SQ>
-__global__ void __launch_bounds__(kThreadsSS, 1)
-mla_decode_ss_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
-                     const DecodeParams p)
+__global__ void __launch_bounds__(kThreads, 1)
+mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
+                  const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     Smem sm;
@@ -1287,30 +1014,11 @@ mla_decode_ss_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_co
     if (!decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) return;
     const int warp = threadIdx.x >> 5;
     const int g = blockIdx.x % p.G;
-    if (warp == 0) ss_producer<N, SQ>(p, w, g, sm, &kv_map, &q_map);
-    else if (warp == 1) ss_mma<N, SQ>(p, w, sm, tmem);
-    else ss_softmax<N, SQ>(p, w, g, sm, tmem);
-    decode_teardown<N, SQ>(tmem);
-}
-
-template <int N, int SQ>
-__global__ void __launch_bounds__(kThreadsTV, 1)
-mla_decode_tv_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
-                     const DecodeParams p)
-{
-    extern __shared__ uint8_t smem_raw[];
-    Smem sm;
-    Range w;
-    uint32_t tmem;
-    ptx::griddep_launch_dependents();
-    if (!decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) return;
-    const int warp = threadIdx.x >> 5;
-    const int g = blockIdx.x % p.G;
-    if (warp == 0) tv_producer<N, SQ>(p, w, g, sm, &kv_map, &q_map);
-    else if (warp == 1) tv_s_mma<N, SQ>(p, w, sm, tmem);
-    else if (warp < 6) tv_softmax<N, SQ>(p, w, g, sm, tmem);
-    else if (warp < 10) tv_transposer<N, SQ>(p, w, sm, tmem);
-    else tv_o_mma<N, SQ>(p, w, sm, tmem);
+    if (warp == 0) producer_warp<N, SQ>(p, w, g, sm, &kv_map, &q_map);
+    else if (warp == 1) score_mma_warp<N, SQ>(p, w, sm, tmem);
+    else if (warp < 6) softmax_warps<N, SQ>(p, w, g, sm, tmem);
+    else if (warp < 10) transposer_warps<N, SQ>(p, w, sm, tmem);
+    else output_mma_warp<N, SQ>(p, w, sm, tmem);
     decode_teardown<N, SQ>(tmem);
 }
 
@@ -1528,11 +1236,7 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
         return MLA_ERR_CUDA;
     }
     const int ki = kernel_index<N, SQ>();
-    void (*kernel)(const CUtensorMap, const CUtensorMap, const DecodeParams);
-    if constexpr (Cfg<N, SQ>::TV)
-        kernel = mla_decode_tv_kernel<N, SQ>;
-    else
-        kernel = mla_decode_ss_kernel<N, SQ>;
+    void (*kernel)(const CUtensorMap, const CUtensorMap, const DecodeParams) = mla_decode_kernel<N, SQ>;
     if (!info.attr_set[ki]) {
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -1540,7 +1244,7 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
         g_dev[dev].attr_set[ki] = true;
     }
     prm.ring = R;
-    kernel<<<grid, Cfg<N, SQ>::THREADS, smem, stream>>>(kv_map, q_map, prm);
+    kernel<<<grid, kThreads, smem, stream>>>(kv_map, q_map, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "mla_decode_kernel launch");
     return MLA_OK;
