@@ -94,8 +94,8 @@ template <int N>
 constexpr uint32_t misc_bytes()
 {
     // barriers, max-reduction buffer [4][N], sum buffer [4][N], reference max [N], shift [N],
-    // tmem holder, abort flag
-    return kMiscRedOffset + (4 * N + 4 * N + N + N) * 4 + 16;
+    // tmem holder, abort flag, 2 spare words, transposer scratch [128]
+    return kMiscRedOffset + (4 * N + 4 * N + N + N) * 4 + 16 + 128 * 4;
 }
 
 struct DecodeParams {
@@ -331,6 +331,7 @@ struct Smem {
     uint32_t bars;           // address of barrier 0
     float *red, *lred;       // column-max exchange [4][N], sum exchange [4][N]
     float *mu, *shift;       // reference max [N], its last shift [N]
+    uint32_t scratch;        // shared-window address of 128 words for the transposer's load fences
     uint32_t *tmem_holder;
     volatile int *abort_flag;
     __device__ __forceinline__ uint32_t bar(int i) const { return bars + 8u * i; }
@@ -645,6 +646,23 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                     }
                 }
             };
+            // The slot is released as soon as this warp's loads of it have
+            // returned, so the ring can refill while this warp waits for a
+            // free V^T block.  Each lane stores a value computed from every
+            // load of the block (so the store cannot complete before the
+            // loads do); the arrive, after a proxy fence, orders that store
+            // before the producer's next TMA write to the slot.
+            auto release = [&](uint32_t slot_id, const uint32_t (&r)[64]) {
+                uint32_t x = 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x |= r[4 * i];
+                ptx::st_shared_b32(sm.scratch + 4u * (32u * q + static_cast<uint32_t>(lane)), x);
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::fence_proxy_async_smem();
+                    ptx::mbar_arrive(sm.bar(kBarEmpty + static_cast<int>(slot_id)));
+                }
+            };
             auto store_chunk = [&](uint32_t vb, uint32_t (&r)[64]) {
                 if (valid < kTile) {
                     // tokens past the sequence end: their P is zero, make V^T zero too
@@ -675,15 +693,16 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
             uint32_t slot_a = 0, slot_b = 0;
             if (!(ok = wait_chunk(0, slot_a))) break;
             load_chunk(slot_a, ra);
+            release(slot_a, ra);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint32_t(&cur)[64] = (j & 1) ? rb : ra;
                 uint32_t(&nxt)[64] = (j & 1) ? ra : rb;
-                uint32_t &slot_cur = (j & 1) ? slot_b : slot_a;
                 uint32_t &slot_nxt = (j & 1) ? slot_a : slot_b;
                 if (j < 3) {
                     if (!(ok = wait_chunk(j + 1, slot_nxt))) break;
                     load_chunk(slot_nxt, nxt);
+                    release(slot_nxt, nxt);
                 }
                 // ring block free: the output MMA that read it last is complete
                 const uint32_t vb = v % NVT, vu = v / NVT;
@@ -691,10 +710,6 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                     break;
                 ptx::tc_fence_after();
                 store_chunk(vb, cur);
-                // the stores consumed this block's registers: release this
-                // warp's share of the slot
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(sm.bar(kBarEmpty + static_cast<int>(slot_cur)));
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -949,6 +964,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.shift = sm.mu + N;
     sm.tmem_holder = reinterpret_cast<uint32_t *>(sm.shift + N);
     sm.abort_flag = reinterpret_cast<volatile int *>(sm.tmem_holder + 1);
+    sm.scratch = ptx::smem_addr(sm.tmem_holder + 4);
 
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {

@@ -420,14 +420,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t v)
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v)
 {
-    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_zero16(uint32_t addr)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 }  // namespace ptx
