@@ -104,9 +104,9 @@ def measured_peaks():
 
 
 def attention_kernel_name(s_q: int, H: int) -> str:
-    """The attention kernel the library launches for this shape: N = s_q * H
-    query columns per CTA (64 at most); N <= 32 keeps V^T in TMEM."""
-    return "mla_decode_tv_kernel" if min(s_q * H, 64) <= 32 else "mla_decode_ss_kernel"
+    """The attention kernel instance the library launches for this shape:
+    N = s_q * H query columns per CTA, at most 64."""
+    return f"mla_decode_kernel<{min(s_q * H, 64)},{s_q}>"
 
 
 def roofline(alg_bytes: int, alg_flops: int, seconds: float, peaks) -> dict:

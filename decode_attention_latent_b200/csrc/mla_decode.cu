@@ -219,6 +219,9 @@ mla_metadata_kernel(const int32_t *__restrict__ seqlens, int B, int s_q, int H, 
     __shared__ int warp_sums[32];
     __shared__ int bad_len;
     const int tid = threadIdx.x;
+    // The attention grid may become resident now: it runs its prologue and
+    // then waits for this grid to complete before reading the schedule.
+    ptx::griddep_launch_dependents();
     if (tid == 0) bad_len = 0;
     __syncthreads();
     for (int b = tid; b < B; b += kMetaThreads) {
@@ -287,20 +290,20 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 // Page-table window: lane j returns the physical block of page `first + j`
 // (0 for pages outside [0, npages), and, with an error bit, for entries that
-// do not name a block of the cache).
+// do not name a block of the cache).  The table entry is loaded whenever it
+// lies inside the table row, so the load does not wait for the length.
 __device__ __forceinline__ int load_pages(const int32_t *bt, int first, int npages, const DecodeParams &p, int lane)
 {
     const int idx = first + lane;
+    const int raw = idx < p.max_blocks ? __ldg(bt + idx) : 0;
     int id = 0;
     if (idx < npages) {
         if (idx >= p.max_blocks) {
             atomicOr(p.err, MLA_DEVERR_SEQLEN);
+        } else if (raw < 0 || static_cast<int64_t>(raw) >= p.num_blocks) {
+            atomicOr(p.err, MLA_DEVERR_BLOCK_TABLE);
         } else {
-            id = __ldg(bt + idx);
-            if (id < 0 || static_cast<int64_t>(id) >= p.num_blocks) {
-                atomicOr(p.err, MLA_DEVERR_BLOCK_TABLE);
-                id = 0;
-            }
+            id = raw;
         }
     }
     return id;
@@ -931,25 +934,17 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 }
 
 // ============================================================== kernel
-// Prologue: schedule check, shared-memory carve-up, barrier initialisation
-// and TMEM allocation.  Returns false (uniformly) when this CTA has no work.
+// Prologue: shared-memory carve-up, barrier initialisation and TMEM
+// allocation (none of which reads an input), then -- once the previous grid
+// of the stream has completed, when launched as its programmatic dependent --
+// the schedule check.  Returns false (uniformly) when this CTA has no work;
+// TMEM is allocated either way and released by decode_teardown.
 template <int N, int SQ>
 __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtensorMap *kv_map,
                                              const CUtensorMap *q_map, uint8_t *smem_raw, Smem &sm, Range &w,
                                              uint32_t &tmem)
 {
     using C = Cfg<N, SQ>;
-    const int tuple = blockIdx.x / p.G;
-    const int32_t *hdr = p.sched;
-    if (hdr[1] != kSchedMagic || hdr[2] != p.B || hdr[3] != p.s_q || hdr[4] != p.H ||
-        hdr[5] != p.num_sms || hdr[6] != p.num_tuples || hdr[7] != p.G) {
-        if (threadIdx.x == 0) atomicOr(p.err, MLA_DEVERR_SCHEDULE);
-        return false;
-    }
-    const int32_t *e = p.sched + kSchedHeader + tuple * kSchedEntry;
-    w = Range{e[0], e[1], e[2], e[3], e[4]};
-    if (w.b0 < 0 || w.b0 >= p.B || w.b1 < w.b0 || w.b1 >= p.B) return false;  // no work for this group
-
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
@@ -999,7 +994,19 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     __syncthreads();
     ptx::tc_fence_after();
     tmem = *sm.tmem_holder;
-    return true;
+
+    // Everything below reads inputs that earlier kernels of the stream write.
+    ptx::griddep_wait();
+    const int tuple = blockIdx.x / p.G;
+    const int32_t *hdr = p.sched;
+    if (hdr[1] != kSchedMagic || hdr[2] != p.B || hdr[3] != p.s_q || hdr[4] != p.H ||
+        hdr[5] != p.num_sms || hdr[6] != p.num_tuples || hdr[7] != p.G) {
+        if (threadIdx.x == 0) atomicOr(p.err, MLA_DEVERR_SCHEDULE);
+        return false;
+    }
+    const int32_t *e = p.sched + kSchedHeader + tuple * kSchedEntry;
+    w = Range{e[0], e[1], e[2], e[3], e[4]};
+    return !(w.b0 < 0 || w.b0 >= p.B || w.b1 < w.b0 || w.b1 >= p.B);  // false: no work for this group
 }
 
 template <int N, int SQ>
@@ -1027,14 +1034,15 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
     Range w;
     uint32_t tmem;
     ptx::griddep_launch_dependents();
-    if (!decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) return;
-    const int warp = threadIdx.x >> 5;
-    const int g = blockIdx.x % p.G;
-    if (warp == 0) producer_warp<N, SQ>(p, w, g, sm, &kv_map, &q_map);
-    else if (warp == 1) score_mma_warp<N, SQ>(p, w, sm, tmem);
-    else if (warp < 6) softmax_warps<N, SQ>(p, w, g, sm, tmem);
-    else if (warp < 10) transposer_warps<N, SQ>(p, w, sm, tmem);
-    else output_mma_warp<N, SQ>(p, w, sm, tmem);
+    if (decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) {
+        const int warp = threadIdx.x >> 5;
+        const int g = blockIdx.x % p.G;
+        if (warp == 0) producer_warp<N, SQ>(p, w, g, sm, &kv_map, &q_map);
+        else if (warp == 1) score_mma_warp<N, SQ>(p, w, sm, tmem);
+        else if (warp < 6) softmax_warps<N, SQ>(p, w, g, sm, tmem);
+        else if (warp < 10) transposer_warps<N, SQ>(p, w, sm, tmem);
+        else output_mma_warp<N, SQ>(p, w, sm, tmem);
+    }
     decode_teardown<N, SQ>(tmem);
 }
 
@@ -1260,8 +1268,20 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
         g_dev[dev].attr_set[ki] = true;
     }
     prm.ring = R;
-    kernel<<<grid, kThreads, smem, stream>>>(kv_map, q_map, prm);
-    e = cudaGetLastError();
+    // Programmatic dependent launch: the CTAs may start their prologue while
+    // the previous kernel of the stream (normally the metadata kernel)
+    // finishes; they read no input before griddepcontrol.wait.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, kv_map, q_map, prm);
     if (e != cudaSuccess) return cuda_fail(e, "mla_decode_kernel launch");
     return MLA_OK;
 }
