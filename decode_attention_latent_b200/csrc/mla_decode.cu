@@ -44,6 +44,7 @@
 #include <cstdio>
 #include <cstring>
 #include <climits>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/mla_decode.h"
@@ -68,7 +69,7 @@ constexpr int kSchedEntry = 8;
 constexpr int kSchedMagic = 0x4D4C4144;         // "MLAD"
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kTau = 8.f;                     // log2-domain headroom before the reference max moves
+constexpr float kTau = 32.f;                    // log2-domain headroom before the reference max moves
 constexpr int kMaxVt = 6;                       // V^T blocks TMEM can hold beside O^T and S^T
 
 // Barrier indices inside the "misc" shared-memory region.
@@ -112,6 +113,7 @@ struct DecodeParams {
     int max_pieces;  // workspace capacity in (piece, group) slots
     int64_t num_blocks;
     float scale_log2;
+    int debug_stall_cta;  // test hook: this CTA never loads its first chunk (-1: none)
 };
 
 struct Range {
@@ -481,6 +483,9 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
                     break;
                 }
                 ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarFull + slot), bytes);
+                // Test hook for the bounded waits: the slot is announced but
+                // never loaded, so its consumers' waits run out.
+                if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
                 ptx::tma_load_3d_elect(sm.slot(slot), kv_map, sm.bar(kBarFull + slot), c * 64, 0, phys0);
                 if (live1)
                     ptx::tma_load_3d_elect(sm.slot(slot) + kPageChunkBytes, kv_map, sm.bar(kBarFull + slot), c * 64,
@@ -1477,6 +1482,11 @@ mla_status_t mla_decode_attention(const uint16_t *q, const uint16_t *kv_cache, c
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
     prm.ring = 0;
     prm.max_pieces = wl.pieces;
+    // Test hook (failure detection): MLA_DEBUG_STALL_CTA=k makes CTA k wait
+    // for a load that is never issued; its waits run out after their time
+    // limit and set MLA_DEVERR_TIMEOUT.  Unset in normal use.
+    prm.debug_stall_cta = -1;
+    if (const char *e = getenv("MLA_DEBUG_STALL_CTA")) prm.debug_stall_cta = atoi(e);
     const int grid = prm.num_tuples * sh.G;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 

@@ -2,8 +2,11 @@
 
 Tolerances (from the arithmetic: bf16 inputs, fp32 accumulation, bf16 P and
 output):
-  out  |gpu - ref| <= 1.5e-2 + |ref| / 256   (1.5e-2 absolute plus one bf16
-       ulp of the reference; for |ref| < 0.6 this is the plain 1.5e-2 bound)
+  out  |gpu - ref| <= 1.5e-2 + ulp_bf16(ref)   (1.5e-2 absolute plus one bf16
+       ulp of the reference, 2^(floor(log2|ref|) - 7): the weights P are
+       rounded to bf16 before the output MMA, which alone can move a near
+       one-hot output by up to 2^-9 |V|, and the output itself is rounded to
+       bf16; for |ref| < 0.6 this is within 4e-3 of the plain 1.5e-2 bound)
        and relative RMSE  sqrt(sum (gpu-ref)^2 / sum ref^2) <= 5e-3;
   lse  |gpu - ref| <= 1e-3, and -inf exactly where the reference is -inf.
 Integer work (the schedule) is compared exactly.
@@ -21,9 +24,14 @@ import oracle
 pytestmark = pytest.mark.gpu
 
 ATOL = 1.5e-2
-RTOL = 1.0 / 256.0
 RMSE_MAX = 5e-3
 LSE_ATOL = 1e-3
+
+
+def ulp_bf16(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    return np.exp2(np.floor(np.log2(np.maximum(a, 1e-30))) - 7)
 
 
 @pytest.fixture(scope="module")
@@ -59,7 +67,7 @@ def compare(g_out, g_lse, r_out, r_lse, seqs=None, what=""):
     assert np.all(g_lse[~fin] == -np.inf), f"{what}: empty rows must have lse = -inf"
     assert np.all(g_out[~fin] == 0), f"{what}: empty rows must have out = 0"
     err = np.abs(g_out - r_out)
-    bound = ATOL + RTOL * np.abs(r_out)
+    bound = ATOL + ulp_bf16(r_out)
     worst = np.unravel_index(np.argmax(err - bound), err.shape)
     assert np.all(err <= bound), (f"{what}: out err {err[worst]:.4e} > {bound[worst]:.4e} at {worst} "
                                   f"(gpu {g_out[worst]:.6f} ref {r_out[worst]:.6f})")
