@@ -1053,20 +1053,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
 
 // =============================================================== combine
 // One 128-thread block per output row (b, i, h) of a sequence cut into pieces.
-// The pieces' lse values go to shared memory once; each thread then owns four
-// latent dims and issues its loads of every piece unrolled, so the partials
-// (fresh in L2) are fetched with all loads in flight instead of one piece at a
-// time.  Launched as a programmatic dependent of the attention kernel: it may
+// Each thread owns four latent dims and issues the loads of a batch of pieces
+// together, so the partials are fetched with all loads in flight instead of
+// one piece at a time; 64 registers a thread keep 8 blocks resident per SM.  Launched as a programmatic dependent of the attention kernel: it may
 // become resident early and waits in hardware for that grid to finish.
 constexpr int kCombineThreads = 128;
 
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 8)
 mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restrict__ ws_o,
                    const float *__restrict__ ws_lse, int B, int s_q, int H, int HG, int G, int max_pieces,
                    uint16_t *__restrict__ out, float *__restrict__ lse, int32_t *__restrict__ err)
 {
-    constexpr int kBatch = 16;  // pieces whose loads are in flight together
-    ptx::griddep_wait();        // the attention grid (and its memory) is complete
+    constexpr int kBatch = 8;  // pieces whose loads are in flight together
+    ptx::griddep_wait();       // the attention grid (and its memory) is complete
     const int tid = threadIdx.x;
     const int64_t r = blockIdx.x;
     const int h = static_cast<int>(r % H);
@@ -1088,34 +1087,41 @@ mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restri
     const int g = h / HG, hl = h % HG;
     const int64_t row0 = (static_cast<int64_t>(first) * G + g) * s_q * HG + static_cast<int64_t>(i) * HG + hl;
     const int64_t pstride = static_cast<int64_t>(G) * s_q * HG;  // rows between consecutive pieces
-    const float *lsrc = ws_lse + row0;
-    const float4 *src = reinterpret_cast<const float4 *>(ws_o + row0 * kDV) + tid;
-    const int64_t step = pstride * kDV / 4;  // float4s between consecutive pieces
-    // Every thread reads all piece lse values itself (broadcast loads) together
-    // with its own partials, so the merge costs one round trip per batch.
-    float M = -INFINITY;
-    for (int k = 0; k < n; ++k) M = fmaxf(M, lsrc[k * pstride]);
-    if (M == -INFINITY) {  // every piece saw no token
-        *o = make_uint2(0, 0);
-        if (tid == 0) lse[r] = -INFINITY;
-        return;
-    }
+    const int64_t step = pstride * kDV / 4;                      // float4s between consecutive pieces
+    const float *lp = ws_lse + row0;
+    const float4 *sp = reinterpret_cast<const float4 *>(ws_o + row0 * kDV) + tid;
+    // Every thread reads the pieces' lse values itself (broadcast loads) with
+    // its own partials, a batch at a time, and keeps a running max, so a row
+    // of up to kBatch pieces costs one round trip.
+    float M = -INFINITY, ssum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float ssum = 0.f;
     for (int k0 = 0; k0 < n; k0 += kBatch) {
         float4 x[kBatch];
         float lk[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            lk[u] = -INFINITY;
             if (k0 + u < n) {
-                x[u] = src[(k0 + u) * step];
-                lk[u] = lsrc[(k0 + u) * pstride];
+                x[u] = *sp;
+                lk[u] = *lp;
             }
+            sp += step;
+            lp += pstride;
         }
+        float bm = lk[0];
+#pragma unroll
+        for (int u = 1; u < kBatch; ++u) bm = fmaxf(bm, lk[u]);
+        if (bm > M) {  // new running max: rescale what was summed so far
+            const float a = (M == -INFINITY) ? 0.f : expf(M - bm);
+            acc.x *= a; acc.y *= a; acc.z *= a; acc.w *= a;
+            ssum *= a;
+            M = bm;
+        }
+        if (M == -INFINITY) continue;  // no piece so far saw a token
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             if (k0 + u < n) {
-                const float wk = expf(lk[u] - M);
+                const float wk = expf(lk[u] - M);  // pieces without tokens: lse = -inf, weight 0
                 ssum += wk;
                 acc.x += wk * x[u].x;
                 acc.y += wk * x[u].y;
@@ -1123,6 +1129,11 @@ mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restri
                 acc.w += wk * x[u].w;
             }
         }
+    }
+    if (M == -INFINITY) {  // every piece saw no token
+        *o = make_uint2(0, 0);
+        if (tid == 0) lse[r] = -INFINITY;
+        return;
     }
     const float inv = 1.f / ssum;
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
