@@ -114,7 +114,7 @@ def test_ragged_lengths_all_shapes(dev, orc, s_q, H):
     compare(g_out, g_lse, r_out, r_lse, what=f"ragged s_q={s_q} H={H}")
 
 
-@pytest.mark.parametrize("n_sms", [1, 2, 3, 17, 148, 400])
+@pytest.mark.parametrize("n_sms", [1, 2, 3, 17, 148, 400, 4096])
 def test_forced_split_counts(dev, orc, n_sms):
     lens = [5, 700, 129, 2048, 64]
     inp = mi.small(B=len(lens), s_q=2, H=16, seqlens=lens, seed=200, tail_fill=float("nan"))
@@ -122,6 +122,28 @@ def test_forced_split_counts(dev, orc, n_sms):
     assert err == 0
     r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
     compare(g_out, g_lse, r_out, r_lse, what=f"num_sms={n_sms}")
+
+
+def test_largest_batch(dev, orc):
+    """4096 sequences (the library's batch limit) of 0..300 tokens, checked on
+    a sample of sequences that includes an empty one and the longest one."""
+    lens = [int(x) for x in np.random.default_rng(11).integers(0, 301, 4096)]
+    lens[7] = 0
+    inp = mi.small(B=4096, s_q=1, H=16, seqlens=lens, seed=1100, tail_fill=float("nan"))
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev)
+    assert err == 0
+    seqs = sorted({0, 7, int(np.argmax(lens)), 4095} | set(int(x) for x in np.random.default_rng(12).integers(0, 4096, 24)))
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale, seqs=seqs)
+    compare(g_out, g_lse, r_out, r_lse, seqs=seqs, what="B=4096")
+
+
+def test_longest_context(dev, orc):
+    """One 256K-token sequence (4096 pages), split over every SM."""
+    inp = mi.small(B=1, s_q=2, H=16, seqlens=[262144], seed=1200)
+    g_out, g_lse, err, _, _ = run_gpu(inp, dev)
+    assert err == 0
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what="L=256K")
 
 
 def test_empty_sequences(dev, orc):
