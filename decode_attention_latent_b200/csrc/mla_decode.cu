@@ -770,7 +770,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         const int te = min((b == w.b1) ? w.t1 : nt, nt);
         if (tb >= te) continue;
         const int split = (b == w.b0) ? w.split0 : 0;
-        const int nvis0 = max(0, L - SQ + 1);  // tokens visible to query position 0
+        const int nvis0 = L - SQ + 1;  // query position i sees tokens < nvis0 + i (none when that is <= 0)
         float l[NG][2], mu[NG][2];             // this thread's columns: running sums, reference max
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) l[gi][0] = l[gi][1] = mu[gi][0] = mu[gi][1] = 0.f;
@@ -803,8 +803,11 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int tok = tok0 + 16 * hf + 8 * (j >> 1);
-                        const int n = 8 * gi + c2 + (j & 1);
-                        const bool vis = (SQ == 2 && n >= HG) ? (tok < L) : (tok < nvis0);
+                        // column n = 8 gi + c2 + (j & 1) belongs to query position
+                        // (8 gi) / HG (HG is a multiple of 8), which sees the first
+                        // L - SQ + 1 + i tokens
+                        const int qi = (8 * gi) / HG;
+                        const bool vis = tok < nvis0 + qi;
                         const float s = __uint_as_float(raw[hf][4 * gi + j]);
                         d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, -mu[gi][j & 1]) : NEG_INF;
                         flag = flag || (d[hf][gi][j] > kTau);
@@ -1152,9 +1155,11 @@ struct Shape {
     int N, SQ, HG, G;
 };
 
+// Query columns per CTA: N = s_q H when that is at most 64, else 64 in
+// G = s_q H / 64 head groups of 64 / s_q heads.
 bool resolve(int s_q, int H, Shape *s)
 {
-    if (s_q != 1 && s_q != 2) return false;
+    if (s_q != 1 && s_q != 2 && s_q != 4 && s_q != 8) return false;
     if (H != 16 && H != 32 && H != 64 && H != 128) return false;
     const int tot = s_q * H;
     s->SQ = s_q;
@@ -1230,7 +1235,9 @@ int kernel_index()
     if (N == 32 && SQ == 1) return 1;
     if (N == 32 && SQ == 2) return 2;
     if (N == 64 && SQ == 1) return 3;
-    return 4;
+    if (N == 64 && SQ == 2) return 4;
+    if (N == 64 && SQ == 4) return 5;
+    return 6;
 }
 
 template <int N, int SQ>
@@ -1506,7 +1513,9 @@ mla_status_t mla_decode_attention(const uint16_t *q, const uint16_t *kv_cache, c
     else if (sh.N == 32 && s_q == 1) rc = launch_decode<32, 1>(kv_map, q_map, prm, grid, st);
     else if (sh.N == 32) rc = launch_decode<32, 2>(kv_map, q_map, prm, grid, st);
     else if (s_q == 1) rc = launch_decode<64, 1>(kv_map, q_map, prm, grid, st);
-    else rc = launch_decode<64, 2>(kv_map, q_map, prm, grid, st);
+    else if (s_q == 2) rc = launch_decode<64, 2>(kv_map, q_map, prm, grid, st);
+    else if (s_q == 4) rc = launch_decode<64, 4>(kv_map, q_map, prm, grid, st);
+    else rc = launch_decode<64, 8>(kv_map, q_map, prm, grid, st);
     return rc;
 }
 

@@ -46,8 +46,11 @@
  *     sched_meta, skips or substitutes the access, and finishes; read it back
  *     with mla_get_device_error.
  *
- * Supported shapes: s_q in {1, 2}; H in {16, 32, 64, 128}; page size 64;
- * head widths 576 / 512; 1 <= B <= 4096; 1 <= num_sms <= 4096.
+ * Supported shapes: s_q in {1, 2, 4, 8}; H in {16, 32, 64, 128}; page size 64;
+ * head widths 576 / 512; 1 <= B <= 4096; 1 <= num_sms <= 4096 and at least
+ * the number of head groups, max(1, s_q * H / 64).  Query position i of an
+ * s_q-token query sees the first seqlen - s_q + 1 + i cached tokens (none
+ * when that is <= 0).
  */
 #ifndef MLA_DECODE_H
 #define MLA_DECODE_H

@@ -152,6 +152,30 @@ def pin_torch_sdpa(orc):
             _close(lse[b, i], torch.logsumexp(scores, dim=-1).numpy(), what=f"lse b={b} i={i}")
 
 
+def pin_torch_sdpa_four_queries(orc):
+    """As pin_torch_sdpa with s_q = 4: query i sees the first seqlen - 3 + i
+    rows, none when that is <= 0 (lengths 1 and 2 leave some queries empty)."""
+    lens = [1, 2, 3, 4, 70, 129]
+    inp = mi.small(B=len(lens), s_q=4, H=2, seqlens=lens, seed=27)
+    out, lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    q = torch.from_numpy(_bf16_to_f64(inp.q))
+    for b, L in enumerate(lens):
+        rows = torch.from_numpy(_rows_of(inp, b, L))
+        for i in range(4):
+            n = max(0, L - 3 + i)
+            if n == 0:
+                assert np.all(out[b, i] == 0) and np.all(np.isneginf(lse[b, i])), "empty context"
+                continue
+            k = rows[:n].unsqueeze(0)
+            v = rows[:n, :512].unsqueeze(0)
+            qq = q[b, i].unsqueeze(1)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qq, k.expand(2, n, 576), v.expand(2, n, 512), scale=inp.scale)
+            _close(out[b, i], ref[:, 0].numpy(), what=f"sdpa4 b={b} i={i}")
+            scores = inp.scale * (qq[:, 0] @ rows[:n].T)
+            _close(lse[b, i], torch.logsumexp(scores, dim=-1).numpy(), what=f"lse4 b={b} i={i}")
+
+
 def pin_causal_rule(orc):
     """Query 0 of an s_q = 2 call equals an s_q = 1 call on seqlen - 1 tokens
     with the same query row; query 1 equals an s_q = 1 call on seqlen tokens."""
@@ -252,6 +276,7 @@ ALL_PINS = [
     pin_weights_sum_to_one,
     pin_two_token_closed_form,
     pin_torch_sdpa,
+    pin_torch_sdpa_four_queries,
     pin_causal_rule,
     pin_paging_invariance,
     pin_tail_rows_unread,

@@ -93,7 +93,7 @@ def test_combine_rejects_bad_arguments(lib):
     assert lib.mla_decode_combine(*bad) == 1
     bad = list(args); bad[3] = 16
     assert lib.mla_decode_combine(*bad) == 4
-    bad = list(args); bad[5] = 4
+    bad = list(args); bad[5] = 3  # s_q = 3 is outside the supported set
     assert lib.mla_decode_combine(*bad) == 3
 
 

@@ -105,7 +105,8 @@ def test_workload_parity(dev, orc, name):
 RAGGED = [1, 63, 64, 65, 127, 128, 129, 1000]
 
 
-@pytest.mark.parametrize("s_q,H", [(1, 16), (1, 32), (1, 64), (1, 128), (2, 16), (2, 32), (2, 64), (2, 128)])
+@pytest.mark.parametrize("s_q,H", [(1, 16), (1, 32), (1, 64), (1, 128), (2, 16), (2, 32), (2, 64), (2, 128),
+                                   (4, 16), (4, 32), (8, 16), (8, 128)])
 def test_ragged_lengths_all_shapes(dev, orc, s_q, H):
     inp = mi.small(B=len(RAGGED), s_q=s_q, H=H, seqlens=RAGGED, seed=100 + H + s_q, tail_fill=float("nan"))
     g_out, g_lse, err, _, _ = run_gpu(inp, dev)
@@ -193,6 +194,21 @@ def test_causal_query0_matches_shorter_context(dev):
     single = run_gpu(one, dev)
     compare(two[0][:, :1], two[1][:, :1], single[0].astype(np.float64), single[1].astype(np.float64),
             what="query 0 vs shorter context")
+
+
+@pytest.mark.parametrize("s_q,H", [(4, 16), (8, 16)])
+def test_causal_every_query_position(dev, s_q, H):
+    """Query position i of an s_q-token call equals a one-token call (another
+    kernel instance) on the first seqlen - s_q + 1 + i tokens."""
+    lens = [2, 130, 3000]
+    inp = mi.small(B=len(lens), s_q=s_q, H=H, seqlens=lens, seed=710 + s_q)
+    multi = run_gpu(inp, dev)
+    for i in range(s_q):
+        one = mi.Inputs(q=inp.q[:, i:i + 1].contiguous(), kv_cache=inp.kv_cache, block_table=inp.block_table,
+                        cache_seqlens=(inp.cache_seqlens - (s_q - 1 - i)).clamp(min=0), scale=inp.scale)
+        single = run_gpu(one, dev)
+        compare(multi[0][:, i:i + 1], multi[1][:, i:i + 1], single[0].astype(np.float64),
+                single[1].astype(np.float64), what=f"s_q={s_q} query {i} vs shorter context")
 
 
 def test_bad_block_table_sets_error_word(dev):
