@@ -32,12 +32,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
 // True once the phase with the given parity has completed.  The waiting
 // thread is parked by the hardware (not spinning) for up to `suspend_ns`
 // while the phase is incomplete, so idle waiters leave the issue slots of
@@ -59,26 +53,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int32_t c0, int32_t c1)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int32_t c0, int32_t c1, int32_t c2)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
@@ -109,26 +83,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05 operation this thread issued before
-// has completed.
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
 
 // 32 lanes x 16 consecutive 32-bit columns: thread t of the warp receives
 // lane (base lane + t), columns col .. col+15.
@@ -161,17 +115,10 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
         : "memory");
 }
 
-// 16 lanes x 256 bits: thread t writes lane (base + t/4) columns 2(t%4), 2(t%4)+1
-// from r0, r1 and lane (base + 8 + t/4), same columns, from r2, r3.
-__device__ __forceinline__ void tmem_st_16x256b(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3)
-{
-    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r0), "r"(r1),
-                 "r"(r2), "r"(r3)
-                 : "memory");
-}
-
-// Four repetitions of the 16x256b pattern along the columns: registers
-// 4k..4k+3 go to columns 8k..8k+7.
+// The 16x256b pattern covers 16 lanes x 256 bits: thread t holds lane
+// (base + t/4) columns 2(t%4), 2(t%4)+1 in r0, r1 and lane (base + 8 + t/4),
+// same columns, in r2, r3.  The .x4 form repeats it four times along the
+// columns: registers 4k..4k+3 go to columns 8k..8k+7.
 __device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -182,7 +129,7 @@ __device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_
         : "memory");
 }
 
-// Loads in the same 16x256b pattern, repeated along the columns: registers
+// Loads in the 16x256b pattern, repeated along the columns: registers
 // 4k..4k+3 come from columns 8k..8k+7 (lane base + t/4: r0, r1; lane
 // base + 8 + t/4: r2, r3).
 __device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t (&r)[8])
@@ -281,6 +228,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 // registers.  The issuing warp therefore runs its loop converged, computes
 // every operand warp-uniformly, and lets elect.sync pick the one lane that
 // executes the instruction.
+// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate;
+// `accumulate` = 0 overwrites D.
 __device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                   uint32_t idesc, uint32_t accumulate)
 {
@@ -307,6 +256,8 @@ __device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tm
         : "memory");
 }
 
+// Arrive once on `bar` when every tcgen05 operation this thread issued before
+// has completed.
 __device__ __forceinline__ void mma_commit_elect(uint32_t bar)
 {
     asm volatile(
@@ -323,15 +274,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32
         "elect.sync r|e, 0xffffffff;\n\t"
         "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}\n" ::"r"(bar),
         "r"(bytes)
-        : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_elect(uint32_t bar)
-{
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|e, 0xffffffff;\n\t"
-        "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}\n" ::"r"(bar)
         : "memory");
 }
 
