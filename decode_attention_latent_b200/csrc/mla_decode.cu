@@ -7,9 +7,9 @@
 //                        contiguous ranges, one per CTA group.
 //   mla_decode_kernel    one persistent CTA per SM.  Per 128-token tile:
 //                          TMA gathers the tile's two pages through the page
-//                          table into a ring of 16 KB shared-memory slots
-//                          (one slot = 64 columns of 128 rows, 128-byte
-//                          swizzled);
+//                          table into a ring of shared-memory slots of one
+//                          or two 16 KB chunks (a chunk = 64 columns of the
+//                          128 rows, 128-byte swizzled);
 //                          S^T = K Q^T on the tensor core (M = 128 tokens,
 //                          N = heads x query positions, K = 576) into TMEM;
 //                          a column-wise online softmax of S^T (running max
@@ -57,11 +57,11 @@ constexpr int kDV = MLA_D_V;
 constexpr int kPage = MLA_PAGE;
 constexpr int kTile = MLA_TILE;
 constexpr int kChunks = kDQK / 64;              // 9 column chunks per row
-constexpr uint32_t kSlotBytes = 16384;          // 128 rows x 128 B
+constexpr uint32_t kChunkBytes = 16384;         // one 64-column chunk of a tile: 128 rows x 128 B
 constexpr uint32_t kPageChunkBytes = 8192;      // 64 rows x 128 B
 constexpr int kThreads = 352;                   // producer, score MMA, 4 softmax, 4 transposer, output MMA
 constexpr int kMaxRing = 16;
-constexpr int kMinRing = 4;                     // the transposer may hold two chunks while the third lands
+constexpr int kMinRingChunks = 4;               // the transposer may hold two chunks while the third lands
 constexpr int kMaxBatch = 4096;
 constexpr int kMaxSms = 4096;
 constexpr int kSchedHeader = 16;
@@ -329,10 +329,27 @@ struct Cfg {
     static constexpr int NVT = (512 - static_cast<int>(VT_COL)) / 64;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(NVT >= 3 && NVT <= kMaxVt, "V^T ring does not fit");
+    // Chunks per ring slot.  One slot is one barrier pair and one producer
+    // round; the loads of a slot (two 8 KB boxes per chunk) are issued back to
+    // back.  Measured on the 16-column shape, 2-chunk slots stream the cache
+    // faster than 1-chunk slots (1.5 us of 108 at a 64K context); at 32
+    // columns they made no difference, and at 64 columns, whose ring is the
+    // smallest, rounding the ring down to whole 2- or 3-chunk slots cost 30
+    // and 60 us.
+    static constexpr int CPS = N == 16 ? 2 : 1;
+    static constexpr int SPT = (kChunks + CPS - 1) / CPS;   // slot uses per tile
+    static constexpr uint32_t SLOT_BYTES = CPS * kChunkBytes;
+    // Arrivals that free a slot: the score MMA's commit and two transposer
+    // warps per latent chunk; the score MMA stands in for the transposer on
+    // the rope chunk (and on the unused chunk positions of the last slot).
+    static constexpr int EMPTY_ARRIVALS = 1 + 2 * CPS;
+    static constexpr int LAST_SLOT_COMMITS = 1 + 2 * (CPS - (kChunks - 1 - (SPT - 1) * CPS));
+    static_assert(CPS >= 1 && CPS <= 3, "chunks per slot");
 };
 
 struct Smem {
     uint32_t ring, q, p;     // shared-window addresses: slot ring, Q, P^T buffers
+    uint32_t slot_bytes;     // bytes per ring slot
     uint32_t bars;           // address of barrier 0
     float *red, *lred;       // column-max exchange [4][N], sum exchange [4][N]
     float *mu, *shift;       // reference max [N], its last shift [N]
@@ -340,7 +357,7 @@ struct Smem {
     uint32_t *tmem_holder;
     volatile int *abort_flag;
     __device__ __forceinline__ uint32_t bar(int i) const { return bars + 8u * i; }
-    __device__ __forceinline__ uint32_t slot(int s) const { return ring + kSlotBytes * s; }
+    __device__ __forceinline__ uint32_t slot(int s) const { return ring + slot_bytes * s; }
 };
 
 // Output of one range: the column sums of the four softmax warps are reduced,
@@ -438,7 +455,7 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     using C = Cfg<N, SQ>;
     const int lane = threadIdx.x & 31;
     const uint32_t R = static_cast<uint32_t>(p.ring);
-    uint32_t cc = 0;  // chunk-slot uses so far
+    uint32_t cc = 0;  // ring slot uses so far
     int qi = 0;       // Q loads so far
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
@@ -474,24 +491,30 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
             const bool live1 = (t * kTile + kPage) < L;
             const uint32_t bytes = live1 ? 2 * kPageChunkBytes : kPageChunkBytes;
 #pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) {
-                const uint32_t u = cc + c;
+            for (int s = 0; s < C::SPT; ++s) {
+                const uint32_t u = cc + s;
                 const int slot = static_cast<int>(u % R);
                 if (!warp_wait(sm.bar(kBarEmpty + slot), ((u / R) & 1) ^ 1, sm.abort_flag, p.err)) {
                     ok = false;
-                    cc += c;  // uses issued so far in this tile
+                    cc += s;  // uses issued so far in this tile
                     break;
                 }
-                ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarFull + slot), bytes);
+                const int c0 = s * C::CPS, c1 = min(c0 + C::CPS, kChunks);
+                ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarFull + slot), bytes * (c1 - c0));
                 // Test hook for the bounded waits: the slot is announced but
                 // never loaded, so its consumers' waits run out.
                 if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
-                ptx::tma_load_3d_elect(sm.slot(slot), kv_map, sm.bar(kBarFull + slot), c * 64, 0, phys0);
-                if (live1)
-                    ptx::tma_load_3d_elect(sm.slot(slot) + kPageChunkBytes, kv_map, sm.bar(kBarFull + slot), c * 64,
-                                           0, phys1);
+                const uint32_t dst = sm.slot(slot);
+#pragma unroll 1
+                for (int c = c0; c < c1; ++c) {
+                    const uint32_t d = dst + (c - c0) * kChunkBytes;
+                    ptx::tma_load_3d_elect(d, kv_map, sm.bar(kBarFull + slot), c * 64, 0, phys0);
+                    if (live1)
+                        ptx::tma_load_3d_elect(d + kPageChunkBytes, kv_map, sm.bar(kBarFull + slot), c * 64, 0,
+                                               phys1);
+                }
             }
-            if (ok) cc += kChunks;
+            if (ok) cc += C::SPT;
         }
     }
     if (!ok) {
@@ -529,29 +552,33 @@ __device__ void score_mma_warp(const DecodeParams &p, const Range &w, const Smem
             const uint32_t d = tmem + C::S_COL + sb * N;
 #pragma unroll 1
             for (int c = 0; c < kChunks; ++c) {
-                const uint32_t u = cc + c;
+                const int s = c / C::CPS, cs = c - s * C::CPS;
+                const uint32_t u = cc + s;
                 const int slot = static_cast<int>(u % R);
-                if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
+                if (cs == 0 && !(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
                 ptx::tc_fence_after();
-                const uint32_t a0 = sm.slot(slot);
+                const uint32_t a0 = sm.slot(slot) + cs * kChunkBytes;
                 const uint32_t b0 = sm.q + c * C::QCHUNK;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     ptx::mma_bf16_ss_elect(d, ptx::desc_sw128(a0 + 32u * k, 16, 1024),
                                            ptx::desc_sw128(b0 + 32u * k, 16, 1024), idS, (c | k) != 0);
-                // a slot is free after three arrivals: this one and one
-                // from each of the two transposer warps that read it; the
-                // rope chunk is not transposed, so it takes all three here
-                ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+                // a slot is free after 1 + 2 CPS arrivals: this commit, once
+                // its last chunk's MMAs are issued, and one from each of the
+                // two transposer warps per latent chunk that read it; the
+                // rope chunk is not transposed, so the last slot takes the
+                // missing arrivals here
                 if (c == kChunks - 1) {
-                    ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+#pragma unroll 1
+                    for (int i = 0; i < C::LAST_SLOT_COMMITS; ++i) ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+                } else if (cs == C::CPS - 1) {
                     ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
                 }
             }
             if (!ok) break;
             ptx::mma_commit_elect(sm.bar(kBarSFull + sb));
             if (t == te - 1) ptx::mma_commit_elect(sm.bar(kBarQEmpty));
-            cc += kChunks;
+            cc += C::SPT;
             ++it;
         }
     }
@@ -636,12 +663,14 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
             // block's loads are issued before this block is stored, so the
             // shared-memory latency is paid about once per block.
             auto wait_chunk = [&](int j, uint32_t &slot_out) -> bool {
-                const uint32_t u = cc + 2 * j + (q >> 1);
+                const int c = 2 * j + (q >> 1);
+                const uint32_t u = cc + c / C::CPS;
                 slot_out = u % R;
                 return warp_wait(sm.bar(kBarFull + static_cast<int>(slot_out)), (u / R) & 1, sm.abort_flag, p.err);
             };
-            auto load_chunk = [&](uint32_t slot_id, uint32_t (&r)[64]) {
-                const uint32_t sbase = sm.slot(static_cast<int>(slot_id));
+            auto load_chunk = [&](int j, uint32_t slot_id, uint32_t (&r)[64]) {
+                const int c = 2 * j + (q >> 1);
+                const uint32_t sbase = sm.slot(static_cast<int>(slot_id)) + (c % C::CPS) * kChunkBytes;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int dc = 32 * (q & 1) + 16 * h + dim_in;  // dim within the chunk
@@ -700,7 +729,7 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
             uint32_t ra[64], rb[64];
             uint32_t slot_a = 0, slot_b = 0;
             if (!(ok = wait_chunk(0, slot_a))) break;
-            load_chunk(slot_a, ra);
+            load_chunk(0, slot_a, ra);
             release(slot_a, ra);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -709,7 +738,7 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                 uint32_t &slot_nxt = (j & 1) ? slot_a : slot_b;
                 if (j < 3) {
                     if (!(ok = wait_chunk(j + 1, slot_nxt))) break;
-                    load_chunk(slot_nxt, nxt);
+                    load_chunk(j + 1, slot_nxt, nxt);
                     release(slot_nxt, nxt);
                 }
                 // ring block free: the output MMA that read it last is complete
@@ -725,7 +754,7 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                 ++v;
             }
             if (!ok) break;
-            cc += kChunks;
+            cc += C::SPT;
         }
     }
 }
@@ -957,9 +986,10 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     sm.ring = base;
-    sm.q = base + p.ring * kSlotBytes;
+    sm.slot_bytes = C::SLOT_BYTES;
+    sm.q = base + p.ring * C::SLOT_BYTES;
     sm.p = sm.q + C::QBYTES;
-    uint8_t *misc = gbase + p.ring * kSlotBytes + C::QBYTES + C::PBYTES;
+    uint8_t *misc = gbase + p.ring * C::SLOT_BYTES + C::QBYTES + C::PBYTES;
     sm.bars = ptx::smem_addr(misc);
     sm.red = reinterpret_cast<float *>(misc + kMiscRedOffset);
     sm.lred = sm.red + 4 * N;
@@ -973,7 +1003,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ring; ++s) {
             ptx::mbar_init(sm.bar(kBarFull + s), 1);
-            ptx::mbar_init(sm.bar(kBarEmpty + s), 3);
+            ptx::mbar_init(sm.bar(kBarEmpty + s), C::EMPTY_ARRIVALS);
         }
         ptx::mbar_init(sm.bar(kBarQFull), 1);
         ptx::mbar_init(sm.bar(kBarQEmpty), 1);
@@ -1245,9 +1275,9 @@ int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
     const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024);
-    int R = (smem_optin - fixed) / static_cast<int>(kSlotBytes);
+    int R = (smem_optin - fixed) / static_cast<int>(C::SLOT_BYTES);
     if (R > kMaxRing) R = kMaxRing;
-    *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * kSlotBytes;
+    *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * C::SLOT_BYTES;
     return R;
 }
 
@@ -1278,8 +1308,8 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
     }
     size_t smem = 0;
     const int R = ring_for<N, SQ>(info.smem_optin, &smem);
-    if (R < kMinRing) {
-        snprintf(g_last_error, sizeof g_last_error, "not enough shared memory for a %d-slot ring", kMinRing);
+    if (R * Cfg<N, SQ>::CPS < kMinRingChunks) {
+        snprintf(g_last_error, sizeof g_last_error, "not enough shared memory for a %d-chunk ring", kMinRingChunks);
         return MLA_ERR_CUDA;
     }
     const int ki = kernel_index<N, SQ>();
