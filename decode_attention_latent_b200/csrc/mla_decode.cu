@@ -290,14 +290,20 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, ok);
 }
 
-// Page-table window: lane j returns the physical block of page `first + j`
-// (0 for pages outside [0, npages), and, with an error bit, for entries that
-// do not name a block of the cache).  The table entry is loaded whenever it
-// lies inside the table row, so the load does not wait for the length.
-__device__ __forceinline__ int load_pages(const int32_t *bt, int first, int npages, const DecodeParams &p, int lane)
+// Page-table window of 32 pages.  table_entry loads lane j's entry for page
+// `first + j` whenever it lies inside the table row, so the load need not
+// wait for the length; checked_page then gives the physical block (0 for
+// pages outside [0, npages), and, with an error bit, for entries that do not
+// name a block of the cache).
+__device__ __forceinline__ int table_entry(const int32_t *bt, int first, const DecodeParams &p, int lane)
 {
     const int idx = first + lane;
-    const int raw = idx < p.max_blocks ? __ldg(bt + idx) : 0;
+    return (idx >= 0 && idx < p.max_blocks) ? __ldg(bt + idx) : 0;
+}
+
+__device__ __forceinline__ int checked_page(int raw, int first, int npages, const DecodeParams &p, int lane)
+{
+    const int idx = first + lane;
     int id = 0;
     if (idx < npages) {
         if (idx >= p.max_blocks) {
@@ -309,6 +315,11 @@ __device__ __forceinline__ int load_pages(const int32_t *bt, int first, int npag
         }
     }
     return id;
+}
+
+__device__ __forceinline__ int load_pages(const int32_t *bt, int first, int npages, const DecodeParams &p, int lane)
+{
+    return checked_page(table_entry(bt, first, p, lane), first, npages, p, lane);
 }
 
 // ================================================================ decode
@@ -459,16 +470,22 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     int qi = 0;       // Q loads so far
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
+        const int tb = (b == w.b0) ? w.t0 : 0;
+        const int32_t *bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks;
+        int win = 2 * tb;
+        // The range's first two page-table windows are fetched together with
+        // the length rather than after it (one memory round trip less before
+        // the first cache load); the entries lie inside the table row, and
+        // only those below the page count are used.
+        const int raw_cur = table_entry(bt, win, p, lane);
+        const int raw_nxt = table_entry(bt, win + 32, p, lane);
         const int L = max(0, __ldg(p.seqlens + b));
         const int nt = tiles_of(L);
-        const int tb = (b == w.b0) ? w.t0 : 0;
         const int te = min((b == w.b1) ? w.t1 : nt, nt);
         if (tb >= te) continue;
-        const int32_t *bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks;
         const int npages = (L + kPage - 1) / kPage;
-        int win = 2 * tb;
-        int cur = load_pages(bt, win, npages, p, lane);
-        int nxt = load_pages(bt, win + 32, npages, p, lane);
+        int cur = checked_page(raw_cur, win, npages, p, lane);
+        int nxt = checked_page(raw_nxt, win + 32, npages, p, lane);
 
         if (!(ok = warp_wait(sm.bar(kBarQEmpty), (qi & 1) ^ 1, sm.abort_flag, p.err))) break;
         ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarQFull), C::QBYTES);
@@ -1044,7 +1061,12 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     }
     const int32_t *e = p.sched + kSchedHeader + tuple * kSchedEntry;
     w = Range{e[0], e[1], e[2], e[3], e[4]};
-    return !(w.b0 < 0 || w.b0 >= p.B || w.b1 < w.b0 || w.b1 >= p.B);  // false: no work for this group
+    if (w.b0 < 0) return false;  // no work for this group
+    if (w.b0 >= p.B || w.b1 < w.b0 || w.b1 >= p.B || w.t0 < 0 || w.t1 < 0) {
+        if (threadIdx.x == 0) atomicOr(p.err, MLA_DEVERR_SCHEDULE);
+        return false;
+    }
+    return true;
 }
 
 template <int N, int SQ>

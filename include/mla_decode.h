@@ -80,7 +80,7 @@ typedef enum {
 /* Bits of the device error word (word 0 of sched_meta). */
 #define MLA_DEVERR_BLOCK_TABLE 1   /* page-table entry outside [0, num_blocks)   */
 #define MLA_DEVERR_SEQLEN 2        /* seqlen < 0 or > max_blocks * 64            */
-#define MLA_DEVERR_SCHEDULE 4      /* sched_meta built for other shapes/num_sms  */
+#define MLA_DEVERR_SCHEDULE 4      /* sched_meta for other shapes, or malformed  */
 #define MLA_DEVERR_TIMEOUT 8       /* a bounded device-side wait ran out         */
 
 /* Length, in int32 words, of the sched_meta buffer for `num_sms` CTAs. */
@@ -112,7 +112,8 @@ mla_status_t mla_decode_metadata(const int32_t *cache_seqlens, int B, int s_q, i
  *   kv_cache       device bf16 [num_blocks, 64, 576], 16-byte aligned.
  *   block_table    device int32 [B, max_blocks]: page p of sequence b lives in
  *                  kv_cache[block_table[b, p]]; entries past a sequence's
- *                  last page are never read.
+ *                  last page are never used (those in the same 32-page
+ *                  window may be loaded, always inside [B, max_blocks]).
  *   cache_seqlens  device int32 [B] (the same buffer given to the metadata).
  *   softmax_scale  finite; applied in fp32 to the scores.
  *   num_sms, sched_meta, num_splits: exactly as produced by

@@ -228,6 +228,21 @@ def test_schedule_for_other_shape_is_detected(dev):
     assert mla.get_device_error(sched) & mla.DEVERR_SCHEDULE
 
 
+def test_malformed_schedule_range_is_detected(dev):
+    # A work range with a negative first tile is refused by the CTA that owns
+    # it (error bit, no page-table or cache access), not followed.
+    inp = mi.small(B=2, s_q=1, H=16, seqlens=[300, 200], seed=802)
+    sl = inp.cache_seqlens.to(dev)
+    sched, splits = mla.decode_metadata(sl, 1, 16, 16)
+    host = sched.cpu()
+    assert host[16] == 0 and host[17] == 0  # group 0 starts at (sequence 0, tile 0)
+    host[17] = -3
+    sched.copy_(host)
+    mla.decode(inp.q.to(dev), inp.kv_cache.to(dev), inp.block_table.to(dev), sl, inp.scale,
+               sched_meta=sched, num_splits=splits, num_sms_=16)
+    assert mla.get_device_error(sched) & mla.DEVERR_SCHEDULE
+
+
 # ---------------------------------------------------- schedule (integers)
 def expected_schedule(lens, tuples):
     tiles = [(max(0, L) + 127) // 128 for L in lens]
