@@ -62,6 +62,8 @@ class Oracle:
         self.lib.mla_oracle_online.restype = ctypes.c_int
         self.lib.mla_oracle_split_merge.argtypes = common + [ctypes.c_int, i64p, f64p, f64p]
         self.lib.mla_oracle_split_merge.restype = ctypes.c_int
+        self.lib.mla_oracle_merge_states.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int64, f64p, f64p]
+        self.lib.mla_oracle_merge_states.restype = ctypes.c_int
         self.lib.mla_oracle_threads.argtypes = []
         self.lib.mla_oracle_threads.restype = ctypes.c_int
 
@@ -154,8 +156,29 @@ class Oracle:
         self._check(rc, "mla_oracle_split_merge")
         return out, lse
 
+    def merge_states(self, out_parts, lse_parts):
+        """Merge W partial states: ``out_parts`` [W, ..., 512], ``lse_parts``
+        [W, ...] (any float dtype, widened exactly to fp64).  Returns fp64
+        (out [..., 512], lse [...])."""
+        o = np.ascontiguousarray(_as_f64(out_parts))
+        l = np.ascontiguousarray(_as_f64(lse_parts))
+        W = o.shape[0]
+        assert o.shape[-1] == 512 and l.shape == o.shape[:-1] and W >= 1
+        rows = int(np.prod(l.shape[1:], dtype=np.int64))
+        out = np.zeros(l.shape[1:] + (512,), dtype=np.float64)
+        lse = np.zeros(l.shape[1:], dtype=np.float64)
+        rc = self.lib.mla_oracle_merge_states(_f64(o), _f64(l), W, rows, _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_merge_states")
+        return out, lse
+
     def threads(self) -> int:
         return int(self.lib.mla_oracle_threads())
+
+
+def _as_f64(t) -> np.ndarray:
+    if hasattr(t, "detach"):  # a torch tensor (bf16 has no numpy dtype: widen through fp32, exactly)
+        t = t.detach().to("cpu").float().numpy()
+    return np.asarray(t, dtype=np.float64)
 
 
 def _f64(a: np.ndarray):

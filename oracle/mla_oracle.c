@@ -45,7 +45,10 @@
  *   mla_oracle_transposed   the transposed flow, as whole matrices per
  *                           sequence: S^T = K Q^T, column softmax, O^T = V^T P^T;
  *   mla_oracle_online       the tiled online-softmax recurrence;
- *   mla_oracle_split_merge  per-range partial results merged through their lse.
+ *   mla_oracle_split_merge  per-range partial results merged through their lse;
+ *   mla_oracle_merge_states the merge step alone, on given partial results
+ *                           (the context-parallel form: each of W ranks
+ *                           attends over its own range of the tokens).
  * They agree to rounding; the tests pin each one to closed forms, library
  * routines and invariants.
  */
@@ -466,4 +469,45 @@ int mla_oracle_split_merge(const uint16_t *q, const uint16_t *kv_cache,
         free(part_o); free(part_lse);
     }
     return failed ? ORC_NO_MEMORY : ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Merge of W partial states of the same output rows, each computed over a   */
+/* disjoint range of the tokens (the last step of mla_oracle_split_merge,     */
+/* taken on its own).  The online softmax of "FlashMLA: compressing the KV    */
+/* cache" (jsqmd.com), "compute flow", step 4, carries a running max and a    */
+/* running sum from one block of keys to the next; merging whole partial      */
+/* results through their log-sum-exps is the same recurrence:                 */
+/*   M = max_w lse_w,  lse = M + ln(sum_w exp(lse_w - M)),                    */
+/*   out = sum_w exp(lse_w - lse) * out_w,                                    */
+/* with out = 0 and lse = -inf when every lse_w is -inf.                      */
+/* out_parts is [W][rows][512], lse_parts [W][rows]; out [rows][512].         */
+/* ------------------------------------------------------------------------ */
+int mla_oracle_merge_states(const double *out_parts, const double *lse_parts, int W, int64_t rows,
+                            double *out, double *lse)
+{
+    if (!out_parts || !lse_parts || !out || !lse || W < 1 || rows < 0) return ORC_BAD_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        double M = -INFINITY;
+        for (int w = 0; w < W; ++w) {
+            const double x = lse_parts[(int64_t)w * rows + r];
+            if (x > M) M = x;
+        }
+        double *o = out + r * ORC_DV;
+        for (int c = 0; c < ORC_DV; ++c) o[c] = 0.0;
+        if (M == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int w = 0; w < W; ++w) sum += exp(lse_parts[(int64_t)w * rows + r] - M);
+        const double total = M + log(sum);
+        for (int w = 0; w < W; ++w) {
+            const double wt = exp(lse_parts[(int64_t)w * rows + r] - total);
+            const double *po = out_parts + ((int64_t)w * rows + r) * ORC_DV;
+            for (int c = 0; c < ORC_DV; ++c) o[c] += wt * po[c];
+        }
+        lse[r] = total;
+    }
+    return ORC_OK;
 }

@@ -269,6 +269,53 @@ def pin_outlier_channels(orc):
         _close(out[0, i], ref[:, 0].numpy(), rel=1e-11, what="outliers")
 
 
+def pin_merge_states_closed_forms(orc):
+    """Merging partial states: one state is returned as it is; two equal
+    states give the same output and lse + ln 2; an empty state (lse = -inf)
+    takes no weight; a row whose states are all empty gives 0 and -inf; lse
+    is torch's logsumexp of the partial lse values."""
+    rng = np.random.default_rng(30)
+    parts = rng.standard_normal((3, 5, 512))
+    lses = rng.standard_normal((3, 5)) * 4
+    out, lse = orc.merge_states(parts[:1], lses[:1])
+    assert np.array_equal(out, parts[0]) and np.array_equal(lse, lses[0])
+    two = np.stack([parts[0], parts[0]])
+    out, lse = orc.merge_states(two, np.stack([lses[0], lses[0]]))
+    _close(out, parts[0], what="two equal states")
+    _close(lse, lses[0] + math.log(2.0), what="two equal states lse")
+    empty = np.array(lses)
+    empty[1] = -np.inf
+    out, lse = orc.merge_states(parts[:2], empty[:2])
+    assert np.array_equal(out, parts[0]) and np.array_equal(lse, lses[0])
+    none = np.full((2, 5), -np.inf)
+    out, lse = orc.merge_states(parts[:2], none)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+    out, lse = orc.merge_states(parts, lses)
+    _close(lse, torch.logsumexp(torch.from_numpy(lses), dim=0).numpy(), what="merged lse vs logsumexp")
+
+
+def pin_merge_states_of_shards_equals_whole(orc):
+    """Attention over page-aligned shards of every sequence (each shard a
+    problem of its own: the same queries, a slice of the page table), merged
+    through the partial lse values, equals attention over the whole
+    sequences; shards past a sequence's end are empty."""
+    lens = [1, 200, 64 * 7 + 5]
+    inp = mi.small(B=3, s_q=1, H=3, seqlens=lens, seed=31)
+    whole = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    cuts = [0, 2, 3, 8]  # page boundaries of three shards
+    outs, lses = [], []
+    for r in range(3):
+        p0, p1 = cuts[r], cuts[r + 1]
+        sl = torch.tensor([min(max(L - 64 * p0, 0), 64 * (p1 - p0)) for L in lens], dtype=torch.int32)
+        bt = inp.block_table[:, p0:p1].contiguous()
+        o, l = orc.direct(inp.q, inp.kv_cache, bt, sl, inp.scale)
+        outs.append(o)
+        lses.append(l)
+    out, lse = orc.merge_states(np.stack(outs), np.stack(lses))
+    _close(out, whole[0], what="merged shards out")
+    _close(lse, whole[1], what="merged shards lse")
+
+
 ALL_PINS = [
     pin_single_token,
     pin_equal_scores_mean_of_values,
@@ -284,4 +331,6 @@ ALL_PINS = [
     pin_online_equals_direct,
     pin_split_merge_equals_unsplit,
     pin_outlier_channels,
+    pin_merge_states_closed_forms,
+    pin_merge_states_of_shards_equals_whole,
 ]

@@ -30,6 +30,13 @@ MUTANTS = [
      "return p->q + (((int64_t)b * p->s_q + i) * p->H + 0) * ORC_DQK;"),
     ("query position ignored", "return p->q + (((int64_t)b * p->s_q + i) * p->H + h) * ORC_DQK;",
      "return p->q + (((int64_t)b * p->s_q + 0) * p->H + h) * ORC_DQK;"),
+    ("merged states weighted by the max, not the total",
+     "const double wt = exp(lse_parts[(int64_t)w * rows + r] - total);",
+     "const double wt = exp(lse_parts[(int64_t)w * rows + r] - M);"),
+    ("merged lse without the max", "        lse[r] = total;\n    }\n    return ORC_OK;",
+     "        lse[r] = log(sum);\n    }\n    return ORC_OK;"),
+    ("merge reads the wrong state's rows", "const double *po = out_parts + ((int64_t)w * rows + r) * ORC_DV;",
+     "const double *po = out_parts + r * ORC_DV;"),
 ]
 
 
