@@ -538,6 +538,90 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_context_parallel_rank(args):
+    """One rank of a W-way context-parallel decode, on one GPU: the decode of
+    this rank's 1/W of every sequence's pages (metadata + attention +
+    combine), then the merge of W partial states.  The all-gather between
+    them (W x B x H x 1028 bytes over NVLink) needs W GPUs and is not timed;
+    its size is reported."""
+    import ctypes
+
+    import decode_attention_latent_b200 as mla
+    from decode_attention_latent_b200.context_parallel import local_shard
+
+    W = args.context_parallel
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lib = mla.load_library()
+    w = mi.WORKLOADS[args.workload]
+    if w.s_q != 1:
+        raise SystemExit("context-parallel decode takes s_q = 1 workloads")
+    inp = mi.make_inputs(w, seed=0)
+    B, H = w.B, w.H
+    sl_h, bt_h = local_shard(inp.cache_seqlens, inp.block_table, W, 0)
+    n_sms = mla.num_sms(dev)
+    q = inp.q.to(dev)
+    n_copies = kv_copy_count(int(sl_h.clamp(min=0).sum()) * 1152, L2_BYTES)
+    kv_copies = [inp.kv_cache.to(dev) for _ in range(min(n_copies, 4))]
+    bt, sl = bt_h.to(dev), sl_h.to(dev)
+    sched = torch.empty(mla.sched_meta_ints(n_sms), dtype=torch.int32, device=dev)
+    splits = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    ws_bytes = mla.workspace_size(B, 1, H, n_sms)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    parts = torch.zeros(W, B, 1, H, mi.D_V, dtype=torch.bfloat16, device=dev)
+    lse_parts = torch.zeros(W, B, 1, H, dtype=torch.float32, device=dev)
+    out = torch.empty(B, 1, H, mi.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    P = ctypes.c_void_p
+
+    def local_decode(kv):
+        assert lib.mla_decode_metadata(P(sl.data_ptr()), B, 1, H, n_sms, P(sched.data_ptr()),
+                                       P(splits.data_ptr()), sp) == 0
+        assert lib.mla_decode(P(q.data_ptr()), P(kv.data_ptr()), P(bt.data_ptr()), P(sl.data_ptr()), B, 1, H,
+                              kv.shape[0], bt.shape[1], ctypes.c_float(inp.scale), n_sms, P(sched.data_ptr()),
+                              P(splits.data_ptr()), P(ws.data_ptr()), ws_bytes, P(parts[0].data_ptr()),
+                              P(lse_parts[0].data_ptr()), sp) == 0
+
+    def merge():
+        assert lib.mla_merge_states(P(parts.data_ptr()), P(lse_parts.data_ptr()), W, B * H, P(out.data_ptr()),
+                                    P(lse.data_ptr()), sp) == 0
+
+    for k in range(max(3, args.warmup)):
+        local_decode(kv_copies[k % len(kv_copies)])
+    parts[1:] = parts[0]
+    lse_parts[1:] = lse_parts[0]
+    for _ in range(max(3, args.warmup)):
+        merge()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev[0].record()
+    for k in range(args.steps):
+        local_decode(kv_copies[k % len(kv_copies)])
+    ev[1].record()
+    ev[2].record()
+    for _ in range(args.steps):
+        merge()
+    ev[3].record()
+    torch.cuda.synchronize(dev)
+    assert mla.get_device_error(sched) == 0
+    dec_us = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
+    mer_us = ev[2].elapsed_time(ev[3]) * 1e3 / args.steps
+    shard_tokens = int(sl_h.sum())
+    line = {
+        "metric": "MLA context-parallel decode us/call per rank (one rank of a W-way length split)",
+        "value": dec_us + mer_us, "unit": "us/call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "W": W, "B": B, "H": H, "shard_tokens_rank0": shard_tokens,
+                   "full_tokens": int(inp.cache_seqlens.sum()), "kv_copies": len(kv_copies)},
+        "decode_us": dec_us, "merge_us": mer_us,
+        "gather_bytes_per_rank": W * B * H * (mi.D_V * 2 + 4),
+        "not_timed": "the all-gather of the W states: one GPU emulates one rank",
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -546,8 +630,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=mi.HEADLINE, choices=sorted(mi.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context-parallel", type=int, default=0, metavar="W",
+                    help="time one rank of a W-way context-parallel decode on one GPU (s_q = 1 workloads)")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
+    if args.context_parallel >= 2 and args.impl == "ours":
+        return run_context_parallel_rank(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_ours(args, world, rank, local)

@@ -41,7 +41,7 @@ DEVERR_TIMEOUT = 8
 EXPORTED = (
     "mla_sched_meta_ints", "mla_decode_workspace_size", "mla_decode_metadata",
     "mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_static_workspace",
-    "mla_get_device_error",
+    "mla_merge_states", "mla_get_device_error",
     "mla_status_string", "mla_last_error_message",
 )
 
@@ -87,6 +87,8 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
     lib.mla_decode_static_workspace.restype = ci
     lib.mla_decode_combine.argtypes = [i32p, i32p, vp, sz, ci, ci, ci, ci, cu16p, vp, vp]
     lib.mla_decode_combine.restype = ci
+    lib.mla_merge_states.argtypes = [cu16p, vp, ci, ctypes.c_int64, cu16p, vp, vp]
+    lib.mla_merge_states.restype = ci
     lib.mla_get_device_error.argtypes = [i32p, ctypes.POINTER(ctypes.c_int32), vp]
     lib.mla_get_device_error.restype = ci
     lib.mla_status_string.argtypes = [ci]
@@ -224,6 +226,35 @@ def decode_combine(num_splits: torch.Tensor, sched_meta: torch.Tensor, workspace
         ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), int(B), int(s_q), int(H), n,
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), _stream_handle(stream, dev))
     _check(rc, "mla_decode_combine")
+
+
+def merge_states(out_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Merge W partial states (``mla_merge_states``): ``out_parts`` bf16
+    [W, ..., 512] and ``lse_parts`` fp32 [W, ...] -> (out bf16 [..., 512],
+    lse fp32 [...])."""
+    dev = out_parts.device
+    if dev.type != "cuda":
+        raise ValueError("out_parts must be a CUDA tensor")
+    if out_parts.dim() < 2 or out_parts.shape[-1] != D_V:
+        raise ValueError(f"out_parts must be [W, ..., {D_V}]")
+    W = out_parts.shape[0]
+    row_shape = tuple(out_parts.shape[1:-1])
+    _require(out_parts, "out_parts", torch.bfloat16, dev)
+    _require(lse_parts, "lse_parts", torch.float32, dev, (W,) + row_shape)
+    if out is None:
+        out = torch.empty(row_shape + (D_V,), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(row_shape, dtype=torch.float32, device=dev)
+    _require(out, "out", torch.bfloat16, dev, row_shape + (D_V,))
+    _require(lse, "lse", torch.float32, dev, row_shape)
+    rows = lse.numel()
+    rc = load_library().mla_merge_states(
+        ctypes.c_void_p(out_parts.data_ptr()), ctypes.c_void_p(lse_parts.data_ptr()), int(W), int(rows),
+        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), _stream_handle(stream, dev))
+    _check(rc, "mla_merge_states")
+    return out, lse
 
 
 def get_device_error(sched_meta: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

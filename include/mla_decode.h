@@ -27,7 +27,10 @@
  *     mla_decode            the attention kernel, then the combine kernel;
  *     mla_decode_attention  the attention kernel alone;
  *     mla_decode_combine    the combine kernel alone (mla_decode already
- *                           launches it; exported for tests and timing).
+ *                           launches it; exported for tests and timing);
+ *     mla_merge_states      context-parallel decode: merges the results of
+ *                           W ranks that each attended over their own range
+ *                           of every sequence's pages.
  *
  * Conventions for every call.
  *   - Pointers marked "device" are CUDA device pointers of the current
@@ -188,6 +191,28 @@ mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_c
                                          float softmax_scale, int num_sms,
                                          const int32_t *sched_meta, const int32_t *num_splits,
                                          uint16_t *out, float *lse, void *stream);
+
+/* Merge of W partial attention states of the same output rows, each computed
+ * over a disjoint range of the tokens -- in context-parallel decode, the
+ * (out, lse) of W ranks that each hold a contiguous range of every sequence's
+ * pages and run mla_decode on it.  The same log-sum-exp merge as the combine
+ * (the online softmax of "FlashMLA: compressing the KV cache", jsqmd.com,
+ * "compute flow", step 4, applied to whole partial results):
+ *     M = max_w lse_w,   lse = M + ln sum_w exp(lse_w - M),
+ *     out = sum_w exp(lse_w - lse) * out_w        (fp32, rounded once to bf16)
+ * with out = 0 and lse = -inf for a row whose states are all empty
+ * (lse_w = -inf, as mla_decode writes for a rank that holds no visible token).
+ *   out_parts   device bf16 [W, rows, 512], 16-byte aligned.
+ *   lse_parts   device fp32 [W, rows] (natural log), 4-byte aligned.
+ *   W           1 <= W <= 64.
+ *   rows        number of output rows, 1 <= rows <= 2^31 - 1 (B * s_q * H
+ *               for decode results).
+ *   out         device bf16 [rows, 512], 16-byte aligned (written).
+ *   lse         device fp32 [rows], 4-byte aligned (written).
+ * Inputs and outputs must not overlap.  Argument errors return before any
+ * launch; asynchronous on `stream`. */
+mla_status_t mla_merge_states(const uint16_t *out_parts, const float *lse_parts, int W, int64_t rows,
+                              uint16_t *out, float *lse, void *stream);
 
 /* Waits for `stream`, copies word 0 of sched_meta to *host_code, and returns
  * MLA_ERR_DEVICE_CHECK if any bit is set (MLA_OK otherwise). */

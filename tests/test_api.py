@@ -100,3 +100,13 @@ def test_combine_rejects_bad_arguments(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(mla.MLAError):
         mla.load_library(str(tmp_path / "missing.so"))
+
+
+def test_merge_states_rejects_bad_arguments(lib):
+    args = [P(GOOD), P(GOOD), 4, 128, P(GOOD), P(GOOD), P(0)]
+    for i, v, status in ((0, P(0), 1), (1, P(0), 1), (4, P(0), 1), (5, P(0), 1), (2, 0, 1), (2, 65, 1),
+                         (3, 0, 1), (3, 1 << 31, 1), (0, P(GOOD + 8), 2), (4, P(GOOD + 8), 2),
+                         (1, P(GOOD + 2), 2), (5, P(GOOD + 1), 2)):
+        bad = list(args)
+        bad[i] = v
+        assert lib.mla_merge_states(*bad) == status, (i, v)
