@@ -421,26 +421,36 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
         write_ok = false;
         piece = 0;
     }
+    // Row n = i HG + hl of the piece is (piece N + n) 512 floats in; of the
+    // final output, ((b SQ + i) H + g HG + hl) 512 bf16.  With the bases and
+    // the per-position stride in registers, each element is one multiply and
+    // one store at a constant offset; up to 32 columns are loaded from TMEM
+    // per wait.  (A range switch at 64 columns spent ~12 us here when every
+    // element recomputed its 64-bit address and each 16 columns waited.)
+    constexpr int CW = N < 32 ? N : 32;
+    float *const wbase = p.ws_o + static_cast<int64_t>(piece) * N * kDV;
+    uint16_t *const obase = p.out + (static_cast<int64_t>(b) * SQ * p.H + g * HG) * kDV;
+    const int64_t ostride = static_cast<int64_t>(p.H) * kDV;  // between query positions
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
         const int dim = j * 128 + row;
 #pragma unroll
-        for (int ch = 0; ch < C::NCH; ++ch) {
-            float v[16];
-            ptx::tmem_ld16(tmem + lane_base + j * N + ch * 16, v);
-            ptx::tmem_wait_ld();
+        for (int c0 = 0; c0 < N; c0 += CW) {
+            float v[CW / 16][16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int n = ch * 16 + e;
-                const int i = n / HG, hl = n % HG;
-                const float val = v[e] * linv[n];
-                if (final_out) {
-                    const int64_t o = ((static_cast<int64_t>(b) * SQ + i) * p.H + g * HG + hl) * kDV + dim;
-                    p.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                } else if (write_ok) {
-                    const int64_t o = ((static_cast<int64_t>(piece) * SQ + i) * HG + hl) * kDV + dim;
-                    p.ws_o[o] = val;
+            for (int k = 0; k < CW / 16; ++k) ptx::tmem_ld16(tmem + lane_base + j * N + c0 + 16 * k, v[k]);
+            ptx::tmem_wait_ld();
+            if (final_out) {
+#pragma unroll
+                for (int e = 0; e < CW; ++e) {
+                    const int n = c0 + e, i = n / HG, hl = n % HG;
+                    obase[i * ostride + hl * kDV + dim] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(v[e / 16][e % 16] * linv[n]));
                 }
+            } else if (write_ok) {
+                float *const wrow = wbase + dim;
+#pragma unroll
+                for (int e = 0; e < CW; ++e) wrow[(c0 + e) * kDV] = v[e / 16][e % 16] * linv[c0 + e];
             }
         }
     }
