@@ -401,15 +401,22 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
         }
     __syncwarp();
     ptx::named_bar_sync(1, 128);
+    // Thread n < N totals column n once: its reciprocal goes to sm.shift (free
+    // between ranges) for every thread, its lse is written below.
+    float ln_own = 0.f;
+    if (tid < N) {
+        ln_own = (sm.lred[tid] + sm.lred[N + tid]) + (sm.lred[2 * N + tid] + sm.lred[3 * N + tid]);
+        sm.shift[tid] = ln_own > 0.f ? 1.f / ln_own : 0.f;
+    }
+    ptx::named_bar_sync(1, 128);
     float linv[N];
 #pragma unroll
     for (int n4 = 0; n4 < N / 4; ++n4) {
-        const float4 *r4 = reinterpret_cast<const float4 *>(sm.lred) + n4;
-        const float4 a0 = r4[0], a1 = r4[N / 4], a2 = r4[2 * (N / 4)], a3 = r4[3 * (N / 4)];
-        const float s[4] = {(a0.x + a1.x) + (a2.x + a3.x), (a0.y + a1.y) + (a2.y + a3.y),
-                            (a0.z + a1.z) + (a2.z + a3.z), (a0.w + a1.w) + (a2.w + a3.w)};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) linv[4 * n4 + e] = s[e] > 0.f ? 1.f / s[e] : 0.f;
+        const float4 a = reinterpret_cast<const float4 *>(sm.shift)[n4];
+        linv[4 * n4 + 0] = a.x;
+        linv[4 * n4 + 1] = a.y;
+        linv[4 * n4 + 2] = a.z;
+        linv[4 * n4 + 3] = a.w;
     }
 
     const int nsplit = p.split_base[b + 1] - p.split_base[b];
@@ -457,7 +464,7 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
     if (tid < N) {
         const int n = tid;
         const int i = n / HG, hl = n % HG;
-        const float ln = (sm.lred[n] + sm.lred[N + n]) + (sm.lred[2 * N + n] + sm.lred[3 * N + n]);
+        const float ln = ln_own;
         const float val = ln > 0.f ? (sm.mu[n] + log2f(ln)) * kLn2 : -INFINITY;
         if (final_out)
             p.lse[(static_cast<int64_t>(b) * SQ + i) * p.H + g * HG + hl] = val;
