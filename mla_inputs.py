@@ -167,6 +167,33 @@ def small(B: int, s_q: int, H: int, seqlens: Sequence[int], table: str = "shuffl
     return make_inputs(w, seed=seed, tail_fill=tail_fill)
 
 
+@dataclass
+class Fp8Cache:
+    """An e4m3 cache with one fp32 scale per cached token (CPU tensors)."""
+    codes: torch.Tensor  # [num_blocks, 64, 576] uint8: e4m3 bit patterns
+    scale: torch.Tensor  # [num_blocks, 64] fp32
+
+
+def fp8_cache(num_blocks: int, seed: int = 0, pow2_scales: bool = False) -> Fp8Cache:
+    """Seeded random e4m3 cache, drawn field by field rather than rounded from
+    real values: sign bits uniform; exponent fields round(N(7, 1.5)) clipped to
+    [0, 14] (magnitudes around 1, subnormals included, no NaN); mantissa fields
+    uniform on 0..7.  Token scales are 2^k, k uniform on {-3, -2, -1}, with
+    ``pow2_scales``, else uniform on [0.05, 0.3).  Draw order: signs,
+    exponents, mantissas, scales."""
+    g = torch.Generator().manual_seed(seed)
+    shape = (num_blocks, PAGE, D_QK)
+    sign = torch.randint(0, 2, shape, generator=g)
+    expo = torch.round(torch.randn(shape, generator=g) * 1.5 + 7.0).clamp(0, 14).to(torch.int64)
+    mant = torch.randint(0, 8, shape, generator=g)
+    codes = ((sign << 7) | (expo << 3) | mant).to(torch.uint8)
+    if pow2_scales:
+        scale = torch.exp2(torch.randint(-3, 0, (num_blocks, PAGE), generator=g).to(torch.float32))
+    else:
+        scale = 0.05 + 0.25 * torch.rand(num_blocks, PAGE, generator=g)
+    return Fp8Cache(codes=codes, scale=scale.to(torch.float32))
+
+
 def algorithmic_bytes(inp: Inputs) -> int:
     """Bytes a decode call must move at minimum: every visible cache row once
     (shared by all heads and query positions), q, out (bf16), lse (fp32) and

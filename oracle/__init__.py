@@ -62,6 +62,12 @@ class Oracle:
         self.lib.mla_oracle_online.restype = ctypes.c_int
         self.lib.mla_oracle_split_merge.argtypes = common + [ctypes.c_int, i64p, f64p, f64p]
         self.lib.mla_oracle_split_merge.restype = ctypes.c_int
+        self.lib.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        self.lib.mla_oracle_e4m3_to_double.restype = ctypes.c_double
+        self.lib.mla_oracle_direct_fp8.argtypes = [u16p, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_float),
+                                                   i32p, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int64, ctypes.c_int, ctypes.c_double, f64p, f64p]
+        self.lib.mla_oracle_direct_fp8.restype = ctypes.c_int
         self.lib.mla_oracle_merge_states.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int64, f64p, f64p]
         self.lib.mla_oracle_merge_states.restype = ctypes.c_int
         self.lib.mla_oracle_threads.argtypes = []
@@ -169,6 +175,32 @@ class Oracle:
         lse = np.zeros(l.shape[1:], dtype=np.float64)
         rc = self.lib.mla_oracle_merge_states(_f64(o), _f64(l), W, rows, _f64(out), _f64(lse))
         self._check(rc, "mla_oracle_merge_states")
+        return out, lse
+
+    def e4m3(self, codes) -> np.ndarray:
+        """Values of e4m3 codes (any integer array), in fp64."""
+        c = np.asarray(codes, dtype=np.uint8)
+        return np.array([self.lib.mla_oracle_e4m3_to_double(int(x)) for x in c.ravel()]).reshape(c.shape)
+
+    def direct_fp8(self, q, kv_codes, kv_scale, block_table, cache_seqlens, scale):
+        """The definition over an e4m3 cache: ``kv_codes`` uint8 [num_blocks, 64,
+        576], ``kv_scale`` fp32 [num_blocks, 64] (one scale per cached token)."""
+        qb = self._bits(q)
+        B, s_q, H, _ = qb.shape
+        codes = np.ascontiguousarray(np.asarray(kv_codes.cpu() if hasattr(kv_codes, "cpu") else kv_codes,
+                                                dtype=np.uint8))
+        ks = np.ascontiguousarray(np.asarray(kv_scale.cpu() if hasattr(kv_scale, "cpu") else kv_scale,
+                                             dtype=np.float32))
+        assert codes.ndim == 3 and codes.shape[1:] == (64, 576) and ks.shape == codes.shape[:2]
+        bt = self._i32(block_table)
+        sl = self._i32(cache_seqlens)
+        out, lse = self._outputs(B, s_q, H)
+        rc = self.lib.mla_oracle_direct_fp8(
+            qb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)), codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+            ks.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), bt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), B, s_q, H, codes.shape[0], bt.shape[1],
+            float(scale), _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_direct_fp8")
         return out, lse
 
     def threads(self) -> int:

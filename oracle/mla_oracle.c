@@ -48,7 +48,9 @@
  *   mla_oracle_split_merge  per-range partial results merged through their lse;
  *   mla_oracle_merge_states the merge step alone, on given partial results
  *                           (the context-parallel form: each of W ranks
- *                           attends over its own range of the tokens).
+ *                           attends over its own range of the tokens);
+ *   mla_oracle_direct_fp8   the definition over an FP8 (e4m3) cache with one
+ *                           fp32 scale per cached token.
  * They agree to rounding; the tests pin each one to closed forms, library
  * routines and invariants.
  */
@@ -510,4 +512,93 @@ int mla_oracle_merge_states(const double *out_parts, const double *lse_parts, in
         lse[r] = total;
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 cache.  The juejin.cn "FlashMLA" post, section 5 (FlashMLA against     */
+/* FlashAttention), says FlashMLA runs in mixed precision such as FP8 and     */
+/* BF16; it fixes no format.  The reading taken here: every cached value is  */
+/* an e4m3 code with one fp32 scale per cached token, so token j's row is     */
+/*   k_j[d] = e4m3(code[blk][j % 64][d]) * kscale[blk][j % 64],  d < 576,     */
+/* and the queries stay bf16.  e4m3 is the OCP FP8 E4M3 format as CUDA's      */
+/* __nv_fp8_e4m3 and torch's float8_e4m3fn hold it: 1 sign, 4 exponent bits  */
+/* (bias 7), 3 mantissa bits, exponent 0 subnormal (mantissa * 2^-9), no     */
+/* infinities, S.1111.111 NaN.  Decoding, and the product with the scale,    */
+/* are exact in double.                                                       */
+/* ------------------------------------------------------------------------ */
+double mla_oracle_e4m3_to_double(uint8_t code)
+{
+    const int sign = code >> 7, ex = (code >> 3) & 15, mant = code & 7;
+    double mag;
+    if (ex == 15 && mant == 7) return NAN;
+    if (ex == 0) mag = ldexp((double)mant, -9);
+    else mag = ldexp(1.0 + mant / 8.0, ex - 7);
+    return sign ? -mag : mag;
+}
+
+int mla_oracle_direct_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                          const int32_t *block_table, const int32_t *seqlens,
+                          int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                          double scale, double *out, double *lse)
+{
+    if (!q || !kv_codes || !kv_scale || !block_table || !seqlens || !out || !lse) return ORC_BAD_ARG;
+    if (B < 0 || s_q < 1 || H < 1 || max_blocks < 1 || num_blocks < 0) return ORC_BAD_ARG;
+    double table[256];
+    for (int c = 0; c < 256; ++c) table[c] = mla_oracle_e4m3_to_double((uint8_t)c);
+    const int64_t rows = (int64_t)B * s_q * H;
+    int failed = 0;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int b = (int)(r / ((int64_t)s_q * H));
+        const int i = (int)((r / H) % s_q);
+        const int h = (int)(r % H);
+        const int64_t n = visible_tokens(seqlens[b] < 0 ? 0 : seqlens[b], s_q, i);
+        double *o = out + r * ORC_DV;
+        for (int c = 0; c < ORC_DV; ++c) o[c] = 0.0;
+        if (n == 0) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double *row = (double *)malloc((size_t)n * ORC_DQK * sizeof(double));
+        double *sc = (double *)malloc((size_t)n * sizeof(double));
+        if (!row || !sc) {
+            failed = 1;
+            free(row); free(sc);
+            continue;
+        }
+        /* dequantised rows of the visible tokens, found through the page table */
+        int bad = 0;
+        for (int64_t j = 0; j < n && !bad; ++j) {
+            const int64_t pg = j / ORC_PAGE;
+            const int32_t blk = pg < max_blocks ? block_table[(int64_t)b * max_blocks + pg] : -1;
+            if (blk < 0 || (int64_t)blk >= num_blocks) { bad = 1; break; }
+            const int64_t tok = (int64_t)blk * ORC_PAGE + j % ORC_PAGE;
+            const double ks = (double)kv_scale[tok];
+            for (int d = 0; d < ORC_DQK; ++d) row[j * ORC_DQK + d] = table[kv_codes[tok * ORC_DQK + d]] * ks;
+        }
+        if (bad) {
+            failed = 2;
+            free(row); free(sc);
+            continue;
+        }
+        const uint16_t *qr = q + r * ORC_DQK;
+        double top = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < ORC_DQK; ++d) acc += bf16_to_double(qr[d]) * row[j * ORC_DQK + d];
+            sc[j] = scale * acc;
+            if (sc[j] > top) top = sc[j];
+        }
+        double total = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            const double wj = exp(sc[j] - top);
+            total += wj;
+            for (int c = 0; c < ORC_DV; ++c) o[c] += wj * row[j * ORC_DQK + c];
+        }
+        for (int c = 0; c < ORC_DV; ++c) o[c] /= total;
+        lse[r] = top + log(total);
+        free(row); free(sc);
+    }
+    return failed == 2 ? ORC_BAD_BLOCK : failed ? ORC_NO_MEMORY : ORC_OK;
 }

@@ -316,6 +316,59 @@ def pin_merge_states_of_shards_equals_whole(orc):
     _close(lse, whole[1], what="merged shards lse")
 
 
+def _e4m3_by_torch(codes) -> np.ndarray:
+    """Library decoding of e4m3 codes: torch's float8_e4m3fn, widened."""
+    c = torch.as_tensor(np.asarray(codes, dtype=np.uint8))
+    return c.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def pin_e4m3_decoding(orc):
+    """Every e4m3 code decodes as torch's float8_e4m3fn does (NaN codes NaN),
+    and spot values of the format: 1.0, 448, 2^-6, 2^-9, -1.0, 0.5, 2.0."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3(codes)
+    ref = _e4m3_by_torch(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and nan.sum() == 2
+    assert np.array_equal(mine[~nan], ref[~nan])
+    spots = {0x38: 1.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0xB8: -1.0, 0x30: 0.5, 0x40: 2.0}
+    for c, v in spots.items():
+        assert orc.e4m3([c])[0] == v, hex(c)
+
+
+def pin_fp8_cache_equals_exact_bf16_cache(orc):
+    """With power-of-two token scales every dequantised value is a bf16 number,
+    so attention over the e4m3 cache equals the (pinned) bf16 definition over
+    that cache dequantised by torch."""
+    inp = mi.small(B=3, s_q=2, H=3, seqlens=[1, 100, 200], seed=33)
+    c = mi.fp8_cache(inp.kv_cache.shape[0], seed=34, pow2_scales=True)
+    deq = torch.from_numpy(_e4m3_by_torch(c.codes.numpy())) * c.scale.to(torch.float64)[..., None]
+    as_bf16 = deq.to(torch.bfloat16)
+    assert torch.equal(as_bf16.to(torch.float64), deq)  # exact in bf16
+    want = orc.direct(inp.q, as_bf16, inp.block_table, inp.cache_seqlens, inp.scale)
+    got = orc.direct_fp8(inp.q, c.codes, c.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    _close(got[0], want[0], what="fp8 out")
+    _close(got[1], want[1], what="fp8 lse")
+
+
+def pin_fp8_cache_against_sdpa(orc):
+    """Arbitrary token scales: torch SDPA in float64 on rows dequantised by
+    torch (float8_e4m3fn times the token's scale)."""
+    inp = mi.small(B=2, s_q=1, H=2, seqlens=[70, 130], seed=35)
+    c = mi.fp8_cache(inp.kv_cache.shape[0], seed=36)
+    out, lse = orc.direct_fp8(inp.q, c.codes, c.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    deq = torch.from_numpy(_e4m3_by_torch(c.codes.numpy())) * c.scale.to(torch.float64)[..., None]
+    q = torch.from_numpy(_bf16_to_f64(inp.q))
+    for b, L in enumerate(inp.cache_seqlens.tolist()):
+        rows = torch.stack([deq[int(inp.block_table[b, j // 64]), j % 64] for j in range(L)])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[b, 0].unsqueeze(1), rows.unsqueeze(0).expand(2, L, 576),
+            rows[:, :512].unsqueeze(0).expand(2, L, 512), scale=inp.scale)
+        _close(out[b, 0], ref[:, 0].numpy(), rel=1e-11, what="fp8 vs sdpa")
+        s = (q[b, 0] @ rows.T) * inp.scale
+        _close(lse[b, 0], torch.logsumexp(s, dim=-1).numpy(), rel=1e-11, what="fp8 lse vs logsumexp")
+
+
 ALL_PINS = [
     pin_single_token,
     pin_equal_scores_mean_of_values,
@@ -333,4 +386,7 @@ ALL_PINS = [
     pin_outlier_channels,
     pin_merge_states_closed_forms,
     pin_merge_states_of_shards_equals_whole,
+    pin_e4m3_decoding,
+    pin_fp8_cache_equals_exact_bf16_cache,
+    pin_fp8_cache_against_sdpa,
 ]

@@ -37,6 +37,12 @@ MUTANTS = [
      "        lse[r] = log(sum);\n    }\n    return ORC_OK;"),
     ("merge reads the wrong state's rows", "const double *po = out_parts + ((int64_t)w * rows + r) * ORC_DV;",
      "const double *po = out_parts + r * ORC_DV;"),
+    ("e4m3 exponent bias off by one", "else mag = ldexp(1.0 + mant / 8.0, ex - 7);",
+     "else mag = ldexp(1.0 + mant / 8.0, ex - 8);"),
+    ("e4m3 subnormals scaled wrongly", "if (ex == 0) mag = ldexp((double)mant, -9);",
+     "if (ex == 0) mag = ldexp((double)mant, -10);"),
+    ("fp8 token scale dropped", "row[j * ORC_DQK + d] = table[kv_codes[tok * ORC_DQK + d]] * ks;",
+     "row[j * ORC_DQK + d] = table[kv_codes[tok * ORC_DQK + d]];"),
 ]
 
 
