@@ -106,7 +106,7 @@ def measured_peaks():
 def attention_kernel_name(s_q: int, H: int) -> str:
     """The attention kernel instance the library launches for this shape:
     N = s_q * H query columns per CTA, at most 64."""
-    return f"mla_decode_kernel<{min(s_q * H, 64)},{s_q}>"
+    return f"mla_decode_kernel<{min(s_q * H, 64)},{s_q},false>"
 
 
 def sustained_tflops() -> float:
@@ -622,6 +622,90 @@ def run_context_parallel_rank(args):
     return 0
 
 
+def run_fp8(args):
+    """The decode over an FP8 (e4m3, one fp32 scale per token) cache of the same
+    workload, one GPU: metadata + attention + combine per call, and the
+    attention kernel alone; its roofline counts 576 + 4 bytes per cached token."""
+    import ctypes
+
+    import decode_attention_latent_b200 as mla
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lib = mla.load_library()
+    w = mi.WORKLOADS[args.workload]
+    if w.s_q != 1 or w.H != 16:
+        raise SystemExit("the FP8 cache path takes s_q = 1, H = 16 workloads")
+    inp = mi.make_inputs(w, seed=0)
+    nb = inp.kv_cache.shape[0]
+    del inp.kv_cache
+    cache = mi.fp8_cache(nb, seed=1)
+    B, H = w.B, w.H
+    n_sms = mla.num_sms(dev)
+    fp8_bytes = nb * 64 * (576 + 4)
+    n_copies = kv_copy_count(fp8_bytes, L2_BYTES)
+    codes = [cache.codes.to(dev) for _ in range(n_copies)]
+    scales = [cache.scale.to(dev) for _ in range(n_copies)]
+    q, bt, sl = inp.q.to(dev), inp.block_table.to(dev), inp.cache_seqlens.to(dev)
+    sched = torch.empty(mla.sched_meta_ints(n_sms), dtype=torch.int32, device=dev)
+    splits = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    ws_bytes = mla.workspace_size(B, 1, H, n_sms)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(B, 1, H, mi.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    P = ctypes.c_void_p
+
+    def meta():
+        assert lib.mla_decode_metadata(P(sl.data_ptr()), B, 1, H, n_sms, P(sched.data_ptr()),
+                                       P(splits.data_ptr()), sp) == 0
+
+    def attn(k):
+        c, s_ = codes[k % n_copies], scales[k % n_copies]
+        assert lib.mla_decode_attention_fp8(P(q.data_ptr()), P(c.data_ptr()), P(s_.data_ptr()), P(bt.data_ptr()),
+                                            P(sl.data_ptr()), B, 1, H, nb, bt.shape[1], ctypes.c_float(inp.scale),
+                                            n_sms, P(sched.data_ptr()), P(splits.data_ptr()), P(ws.data_ptr()),
+                                            ws_bytes, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
+
+    def comb():
+        assert lib.mla_decode_combine(P(splits.data_ptr()), P(sched.data_ptr()), P(ws.data_ptr()), ws_bytes, B, 1, H,
+                                      n_sms, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
+
+    for k in range(max(3, args.warmup)):
+        meta(); attn(k); comb()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(args.steps):
+        meta(); attn(k); comb()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    call_us = e0.elapsed_time(e1) * 1e3 / args.steps
+    meta()
+    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for k in range(args.steps):
+        a_ev[k][0].record(); attn(k); a_ev[k][1].record()
+    torch.cuda.synchronize(dev)
+    assert mla.get_device_error(sched) == 0
+    attn_us = statistics.mean(a.elapsed_time(b) for a, b in a_ev) * 1e3
+    tokens = int(inp.cache_seqlens.sum())
+    alg = tokens * (576 + 4) + q.numel() * 2 + out.numel() * 2 + lse.numel() * 4 + sum(
+        (int(L) + 63) // 64 for L in inp.cache_seqlens.tolist()) * 4
+    hbm = measured_peaks()[0]
+    line = {
+        "metric": "MLA decode us/call over an FP8 (e4m3, per-token scale) cache", "value": call_us, "unit": "us/call",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+        "dtype": "e4m3 cache, bf16 MMA", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "H": H, "cache_copies": n_copies},
+        "attention_us": attn_us,
+        "roofline": {"bound": "hbm", "achieved": alg / (attn_us * 1e-6) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": alg / (attn_us * 1e-6) / 1e9 / hbm, "algorithmic_bytes_per_launch": alg,
+                     "traffic": None},
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -630,12 +714,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=mi.HEADLINE, choices=sorted(mi.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true", help="the same workload over an FP8 (e4m3) cache (H = 16, s_q = 1)")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="W",
                     help="time one rank of a W-way context-parallel decode on one GPU (s_q = 1 workloads)")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
     if args.context_parallel >= 2 and args.impl == "ours":
         return run_context_parallel_rank(args)
+    if args.fp8 and args.impl == "ours":
+        return run_fp8(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_ours(args, world, rank, local)

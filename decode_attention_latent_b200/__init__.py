@@ -41,7 +41,7 @@ DEVERR_TIMEOUT = 8
 EXPORTED = (
     "mla_sched_meta_ints", "mla_decode_workspace_size", "mla_decode_metadata",
     "mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_static_workspace",
-    "mla_merge_states", "mla_get_device_error",
+    "mla_merge_states", "mla_decode_fp8", "mla_decode_attention_fp8", "mla_get_device_error",
     "mla_status_string", "mla_last_error_message",
 )
 
@@ -87,6 +87,11 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
     lib.mla_decode_static_workspace.restype = ci
     lib.mla_decode_combine.argtypes = [i32p, i32p, vp, sz, ci, ci, ci, ci, cu16p, vp, vp]
     lib.mla_decode_combine.restype = ci
+    lib.mla_decode_fp8.argtypes = [cu16p, vp, vp, i32p, i32p, ci, ci, ci, ctypes.c_int64, ci,
+                                   ctypes.c_float, ci, i32p, i32p, vp, sz, cu16p, vp, vp]
+    lib.mla_decode_fp8.restype = ci
+    lib.mla_decode_attention_fp8.argtypes = lib.mla_decode_fp8.argtypes
+    lib.mla_decode_attention_fp8.restype = ci
     lib.mla_merge_states.argtypes = [cu16p, vp, ci, ctypes.c_int64, cu16p, vp, vp]
     lib.mla_merge_states.restype = ci
     lib.mla_get_device_error.argtypes = [i32p, ctypes.POINTER(ctypes.c_int32), vp]
@@ -226,6 +231,55 @@ def decode_combine(num_splits: torch.Tensor, sched_meta: torch.Tensor, workspace
         ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), int(B), int(s_q), int(H), n,
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), _stream_handle(stream, dev))
     _check(rc, "mla_decode_combine")
+
+
+def decode_fp8(q: torch.Tensor, kv_codes: torch.Tensor, kv_scale: torch.Tensor, block_table: torch.Tensor,
+               cache_seqlens: torch.Tensor, softmax_scale: float, *, sched_meta: Optional[torch.Tensor] = None,
+               num_splits: Optional[torch.Tensor] = None, num_sms_: Optional[int] = None,
+               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+               combine: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MLA decode over an FP8 cache (``mla_decode_fp8``): ``kv_codes`` uint8
+    [num_blocks, 64, 576] e4m3 codes, ``kv_scale`` fp32 [num_blocks, 64], one
+    scale per cached token.  s_q = 1, H = 16."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("q must be a CUDA tensor")
+    if q.dim() != 4 or q.shape[-1] != D_QK:
+        raise ValueError(f"q must be [B, s_q, H, {D_QK}]")
+    B, s_q, H, _ = q.shape
+    _require(q, "q", torch.bfloat16, dev)
+    if kv_codes.dim() != 3 or tuple(kv_codes.shape[1:]) != (PAGE, D_QK):
+        raise ValueError(f"kv_codes must be [num_blocks, {PAGE}, {D_QK}]")
+    _require(kv_codes, "kv_codes", torch.uint8, dev)
+    _require(kv_scale, "kv_scale", torch.float32, dev, (kv_codes.shape[0], PAGE))
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_blocks]")
+    _require(block_table, "block_table", torch.int32, dev)
+    _require(cache_seqlens, "cache_seqlens", torch.int32, dev, (B,))
+    n = num_sms(dev) if num_sms_ is None else int(num_sms_)
+    if sched_meta is None or num_splits is None:
+        sched_meta, num_splits = decode_metadata(cache_seqlens, s_q, H, n, stream=stream)
+    ws_bytes = workspace_size(B, s_q, H, n)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty(B, s_q, H, D_V, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+    _require(out, "out", torch.bfloat16, dev, (B, s_q, H, D_V))
+    _require(lse, "lse", torch.float32, dev, (B, s_q, H))
+    lib = load_library()
+    fn = lib.mla_decode_fp8 if combine else lib.mla_decode_attention_fp8
+    rc = fn(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(kv_codes.data_ptr()), ctypes.c_void_p(kv_scale.data_ptr()),
+        ctypes.c_void_p(block_table.data_ptr()), ctypes.c_void_p(cache_seqlens.data_ptr()),
+        B, s_q, H, kv_codes.shape[0], block_table.shape[1], float(softmax_scale), n,
+        ctypes.c_void_p(sched_meta.data_ptr()), ctypes.c_void_p(num_splits.data_ptr()),
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), _stream_handle(stream, dev))
+    _check(rc, "mla_decode_fp8" if combine else "mla_decode_attention_fp8")
+    return out, lse
 
 
 def merge_states(out_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optional[torch.Tensor] = None,

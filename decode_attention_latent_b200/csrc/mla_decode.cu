@@ -85,14 +85,31 @@ constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
 constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
 constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
 constexpr int kBarDrainO = kBarDrain + 1;
-constexpr int kNumBars = kBarDrainO + 1;
+// FP8 cache (16 query columns): a ring of staging units between the TMA and
+// the bf16 chunk ring.  A unit is one 128-column group of the tile's 128 rows
+// in e4m3 (two 8 KB page halves, 128-byte swizzled), then, for a tile's first
+// unit, its 128 token scales; 17 KB keeps every unit 1024-byte aligned.
+constexpr int kF8Ring = 4;
+constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
+constexpr uint32_t kF8Unit = 17408;
+constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B
+constexpr uint32_t kF8ScaleOff = 16384;
+constexpr int kBarF8Full = kBarDrainO + 1;         // [kF8Ring] unit loaded
+constexpr int kBarF8Empty = kBarF8Full + kF8Ring;  // [kF8Ring] unit converted
+// FP8: the token scales of a tile, copied by the converter warps for the
+// softmax (a unit is handed back to the producer before the softmax runs).
+constexpr int kScBufs = 4;
+constexpr uint32_t kScBytes = kScBufs * 128 * 4;
+constexpr int kBarScFull = kBarF8Empty + kF8Ring;  // [kScBufs] scales of a tile written
+constexpr int kBarScEmpty = kBarScFull + kScBufs;  // [kScBufs] scales read by the softmax
+constexpr int kNumBars = kBarScEmpty + kScBufs;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
 constexpr uint32_t kMiscRedOffset = (kNumBars * 8 + 127) / 128 * 128;
 static_assert(kMiscRedOffset % 16 == 0, "reduction buffers must be 16-byte aligned");
 
 template <int N>
-constexpr uint32_t misc_bytes()
+__host__ __device__ constexpr uint32_t misc_bytes()
 {
     // barriers, max-reduction buffer [4][N], sum buffer [4][N], reference max [N], shift [N],
     // tmem holder, abort flag, 2 spare words, transposer scratch [128]
@@ -361,6 +378,8 @@ struct Cfg {
 struct Smem {
     uint32_t ring, q, p;     // shared-window addresses: slot ring, Q, P^T buffers
     uint32_t slot_bytes;     // bytes per ring slot
+    uint32_t f8;             // shared-window address of the FP8 staging ring (FP8 cache only)
+    float *tscale;           // FP8: token scales of kScBufs tiles [kScBufs][128]
     uint32_t bars;           // address of barrier 0
     float *red, *lred;       // column-max exchange [4][N], sum exchange [4][N]
     float *mu, *shift;       // reference max [N], its last shift [N]
@@ -476,14 +495,14 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
 }
 
 // -- producer warp: Q per range, then each tile's 9 chunks in order --------
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, const Smem &sm,
-                              const CUtensorMap *kv_map, const CUtensorMap *q_map)
+                              const CUtensorMap *kv_map, const CUtensorMap *q_map, const CUtensorMap *sc_map)
 {
     using C = Cfg<N, SQ>;
     const int lane = threadIdx.x & 31;
     const uint32_t R = static_cast<uint32_t>(p.ring);
-    uint32_t cc = 0;  // ring slot uses so far
+    uint32_t cc = 0;  // ring slot uses so far (bf16 cache) / staging unit uses so far (FP8 cache)
     int qi = 0;       // Q loads so far
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
@@ -523,6 +542,35 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
             const int phys0 = __shfl_sync(0xffffffffu, cur, 2 * t - win);
             const int phys1 = __shfl_sync(0xffffffffu, cur, 2 * t + 1 - win);
             const bool live1 = (t * kTile + kPage) < L;
+            if constexpr (F8) {
+                // FP8: the tile's five 128-column groups into the staging ring,
+                // the token scales with the first; the transposer warps turn
+                // each unit into one bf16 ring slot.
+                const uint32_t b8 = live1 ? 2 * kF8Half : kF8Half;
+                const uint32_t bsc = live1 ? 512u : 256u;
+#pragma unroll 1
+                for (int k = 0; k < kF8Units; ++k) {
+                    const uint32_t u = cc + k;
+                    const int us = static_cast<int>(u % kF8Ring);
+                    if (!warp_wait(sm.bar(kBarF8Empty + us), ((u / kF8Ring) & 1) ^ 1, sm.abort_flag, p.err)) {
+                        ok = false;
+                        cc += k;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarF8Full + us), b8 + (k == 0 ? bsc : 0u));
+                    if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
+                    const uint32_t dst = sm.f8 + us * kF8Unit;
+                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarF8Full + us), 128 * k, 0, phys0);
+                    if (live1) ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarF8Full + us), 128 * k, 0, phys1);
+                    if (k == 0) {
+                        ptx::tma_load_2d_elect(dst + kF8ScaleOff, sc_map, sm.bar(kBarF8Full + us), 0, phys0);
+                        if (live1)
+                            ptx::tma_load_2d_elect(dst + kF8ScaleOff + 256, sc_map, sm.bar(kBarF8Full + us), 0, phys1);
+                    }
+                }
+                if (ok) cc += kF8Units;
+                continue;
+            }
             const uint32_t bytes = live1 ? 2 * kPageChunkBytes : kPageChunkBytes;
 #pragma unroll 1
             for (int s = 0; s < C::SPT; ++s) {
@@ -553,9 +601,11 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     }
     if (!ok) {
         // Let every load this warp issued land before the CTA exits.
-        const uint32_t first = cc > R ? cc - R : 0;
+        const uint32_t RR = F8 ? static_cast<uint32_t>(kF8Ring) : R;
+        const int full0 = F8 ? kBarF8Full : kBarFull;
+        const uint32_t first = cc > RR ? cc - RR : 0;
         for (uint32_t u = first; u < cc; ++u)
-            warp_wait(sm.bar(kBarFull + static_cast<int>(u % R)), (u / R) & 1, sm.abort_flag, p.err, false);
+            warp_wait(sm.bar(full0 + static_cast<int>(u % RR)), (u / RR) & 1, sm.abort_flag, p.err, false);
     }
 }
 
@@ -667,15 +717,18 @@ __device__ void output_mma_warp(const DecodeParams &p, const Range &w, const Sme
 // Warp q owns TMEM lanes 32q..32q+31, i.e. latent dims 128j + 32q + (0..31)
 // of every 128-dim block j: half of chunk 2j + q/2.  Per 16 dims x 16 tokens
 // one ldmatrix.x4.trans feeds one tcgen05.st.16x256b.
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
     constexpr uint32_t NVT = C::NVT;
+    static_assert(!F8 || C::CPS == 2, "FP8 staging unit = one 2-chunk ring slot");
     const uint32_t R = static_cast<uint32_t>(p.ring);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;
     uint32_t cc = 0, v = 0;
+    uint32_t c8 = 0;         // FP8 staging unit uses so far
+    bool vt_ok = true;       // FP8: a failed V^T wait, carried to the next agreement
     bool ok = true;
     // ldmatrix row addresses: lane -> (matrix mi, row rr).  Matrices 0 and 2
     // take tokens {0,1,4,5,8,9,12,13} of a 16-token group, matrices 1 and 3
@@ -761,6 +814,100 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                     }
             };
             uint32_t ra[64], rb[64];
+            if constexpr (F8) {
+                // Unit k of the tile becomes ring slot cc + k (chunks 2k, 2k + 1;
+                // the rope group fills the first chunk of slot cc + 4): thread
+                // row r converts its token's 128 e4m3 codes to bf16 (exactly),
+                // in the swizzled layout the TMA gives bf16 chunks; then the
+                // slot is handed to the score MMA (full barrier, four warp
+                // arrivals) and the unit back to the producer.  The token's
+                // scale goes to the softmax, which applies it in fp32 to the
+                // token's scores and to its weights in P^T.
+                auto convert = [&](int k) -> bool {
+                    const uint32_t u8 = c8 + k;
+                    const int us = static_cast<int>(u8 % kF8Ring);
+                    if (!warp_wait(sm.bar(kBarF8Full + us), (u8 / kF8Ring) & 1, sm.abort_flag, p.err)) return false;
+                    const uint32_t su = cc + k;
+                    const int slot = static_cast<int>(su % R);
+                    if (!warp_wait(sm.bar(kBarEmpty + slot), ((su / R) & 1) ^ 1, sm.abort_flag, p.err)) return false;
+                    const uint32_t src = sm.f8 + us * kF8Unit;
+                    const uint32_t r = static_cast<uint32_t>(32 * q + lane);
+                    const uint32_t sw = r & 7u;
+                    if (k == 0) {
+                        // this row's token scale, for the softmax of this tile
+                        const uint32_t tile = c8 / kF8Units, sbuf = tile % kScBufs;
+                        if (!warp_wait(sm.bar(kBarScEmpty + sbuf), ((tile / kScBufs) & 1) ^ 1, sm.abort_flag, p.err))
+                            return false;
+                        sm.tscale[sbuf * 128 + r] = ptx::ld_shared_f32(src + kF8ScaleOff + 4u * r);
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(sm.bar(kBarScFull + sbuf));
+                    }
+                    const uint32_t dst = sm.slot(slot) + r * 128u;
+                    const int nlu = (k == kF8Units - 1) ? 4 : 8;  // the rope group is 64 columns
+#pragma unroll
+                    for (int lu = 0; lu < 8; ++lu) {
+                        if (lu < nlu) {
+                            const uint4 wv = ptx::ld_shared_v4(src + r * 128u + ((static_cast<uint32_t>(lu) ^ sw) << 4));
+                            const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                            uint32_t o[8];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float2 lo = ptx::e4m3x2_to_float2(words[i], false);
+                                const float2 hi = ptx::e4m3x2_to_float2(words[i], true);
+                                o[2 * i] = ptx::pack_bf16x2(lo.x, lo.y);  // exact: e4m3 values are bf16 values
+                                o[2 * i + 1] = ptx::pack_bf16x2(hi.x, hi.y);
+                            }
+                            const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
+                            const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
+                            ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
+                            ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                        }
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::mbar_arrive(sm.bar(kBarFull + slot));
+                        ptx::mbar_arrive(sm.bar(kBarF8Empty + us));
+                    }
+                    return true;
+                };
+                const uint32_t s0 = cc % R;
+                // The four converter warps agree (named barrier 2) after every
+                // conversion, so every row of a slot is written before any warp
+                // reads it transposed, and a failed wait ends all four together.
+                bool okc = convert(0);
+                if (!(ok = ptx::named_bar_and(2, 128, okc && vt_ok))) break;
+                load_chunk(0, s0, ra);
+                release(s0, ra);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t(&cur)[64] = (j & 1) ? rb : ra;
+                    uint32_t(&nxt)[64] = (j & 1) ? ra : rb;
+                    if (j < 3) {
+                        okc = convert(j + 1);
+                        if (j == 2) okc = convert(kF8Units - 1) && okc;
+                        if (!(ok = ptx::named_bar_and(2, 128, okc && vt_ok))) break;
+                        const uint32_t sn = (cc + static_cast<uint32_t>(j) + 1u) % R;
+                        load_chunk(j + 1, sn, nxt);
+                        release(sn, nxt);
+                    }
+                    const uint32_t vb = v % NVT, vu = v / NVT;
+                    if (vu >= 1) vt_ok = warp_wait(sm.bar(kBarVtEmpty + vb), (vu & 1) ^ 1, sm.abort_flag, p.err) && vt_ok;
+                    if (vt_ok) {
+                        ptx::tc_fence_after();
+                        store_chunk(vb, cur);
+                        ptx::tmem_wait_st();
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(sm.bar(kBarVtFull + vb));
+                    }
+                    ++v;
+                }
+                if (!ok) break;
+                cc += C::SPT;
+                c8 += kF8Units;
+                continue;
+            }
             uint32_t slot_a = 0, slot_b = 0;
             if (!(ok = wait_chunk(0, slot_a))) break;
             load_chunk(0, slot_a, ra);
@@ -807,7 +954,7 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
 // weights 2^(s - mu) are at most 2^kTau and nothing is rescaled.  Every weight
 // of a column is taken relative to the same mu as its sum, so the result is
 // the same softmax.
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
@@ -857,6 +1004,22 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             // pass 1: masked log2-domain scores relative to mu
             const bool first = (t == tb);
             const int tok0 = t * kTile + 32 * wq + r8;
+            // FP8 cache: the scales of this thread's four token rows (0 for rows
+            // past the visible tokens, so their zero weights stay zero)
+            float tsc[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
+            if constexpr (F8) {
+                const uint32_t sbuf = it % kScBufs;
+                wait_ok = wait_bounded(sm.bar(kBarScFull + sbuf), (it / kScBufs) & 1, sm.abort_flag, p.err) && wait_ok;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int row = 32 * wq + r8 + 16 * hf + 8 * jj;
+                        tsc[hf][jj] = (tok0 + 16 * hf + 8 * jj < nvis0) ? sm.tscale[sbuf * 128 + row] : 0.f;
+                    }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(sm.bar(kBarScEmpty + sbuf));
+            }
             float d[2][NG][4];
             bool flag = first || !wait_ok;
 #pragma unroll
@@ -871,7 +1034,8 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                         // L - SQ + 1 + i tokens
                         const int qi = (8 * gi) / HG;
                         const bool vis = tok < nvis0 + qi;
-                        const float s = __uint_as_float(raw[hf][4 * gi + j]);
+                        float s = __uint_as_float(raw[hf][4 * gi + j]);
+                        if constexpr (F8) s *= tsc[hf][j >> 1];
                         d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, -mu[gi][j & 1]) : NEG_INF;
                         flag = flag || (d[hf][gi][j] > kTau);
                     }
@@ -974,8 +1138,13 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                     const float p3 = ptx::ex2_approx(d[hf][gi][3]);
                     l[gi][0] += p0 + p2;
                     l[gi][1] += p1 + p3;
-                    pk[gi][0] = ptx::pack_bf16x2(p0, p1);  // token row r8
-                    pk[gi][1] = ptx::pack_bf16x2(p2, p3);  // token row r8 + 8
+                    if constexpr (F8) {  // V holds the codes: the token's scale goes with its weight
+                        pk[gi][0] = ptx::pack_bf16x2(p0 * tsc[hf][0], p1 * tsc[hf][0]);
+                        pk[gi][1] = ptx::pack_bf16x2(p2 * tsc[hf][1], p3 * tsc[hf][1]);
+                    } else {
+                        pk[gi][0] = ptx::pack_bf16x2(p0, p1);  // token row r8
+                        pk[gi][1] = ptx::pack_bf16x2(p2, p3);  // token row r8 + 8
+                    }
                 }
                 // P^T rows n, K positions = tokens of the tile (natural order)
                 const int kb = 32 * wq + 16 * hf + 8 * st_blk;  // first token of this lane's matrix
@@ -1010,10 +1179,10 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 // of the stream has completed, when launched as its programmatic dependent --
 // the schedule check.  Returns false (uniformly) when this CTA has no work;
 // TMEM is allocated either way and released by decode_teardown.
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtensorMap *kv_map,
-                                             const CUtensorMap *q_map, uint8_t *smem_raw, Smem &sm, Range &w,
-                                             uint32_t &tmem)
+                                             const CUtensorMap *q_map, const CUtensorMap *sc_map, uint8_t *smem_raw,
+                                             Smem &sm, Range &w, uint32_t &tmem)
 {
     using C = Cfg<N, SQ>;
     const uint32_t raw = ptx::smem_addr(smem_raw);
@@ -1021,9 +1190,12 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     uint8_t *gbase = smem_raw + (base - raw);
     sm.ring = base;
     sm.slot_bytes = C::SLOT_BYTES;
-    sm.q = base + p.ring * C::SLOT_BYTES;
+    uint32_t off = p.ring * C::SLOT_BYTES;
+    sm.f8 = base + off;
+    if constexpr (F8) off += kF8Ring * kF8Unit;
+    sm.q = base + off;
     sm.p = sm.q + C::QBYTES;
-    uint8_t *misc = gbase + p.ring * C::SLOT_BYTES + C::QBYTES + C::PBYTES;
+    uint8_t *misc = gbase + off + C::QBYTES + C::PBYTES;
     sm.bars = ptx::smem_addr(misc);
     sm.red = reinterpret_cast<float *>(misc + kMiscRedOffset);
     sm.lred = sm.red + 4 * N;
@@ -1032,12 +1204,21 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.tmem_holder = reinterpret_cast<uint32_t *>(sm.shift + N);
     sm.abort_flag = reinterpret_cast<volatile int *>(sm.tmem_holder + 1);
     sm.scratch = ptx::smem_addr(sm.tmem_holder + 4);
+    sm.tscale = reinterpret_cast<float *>(misc + misc_bytes<N>());  // FP8 only: kScBytes past the misc region
 
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ring; ++s) {
-            ptx::mbar_init(sm.bar(kBarFull + s), 1);
+            ptx::mbar_init(sm.bar(kBarFull + s), F8 ? 4 : 1);  // FP8: the four converter warps
             ptx::mbar_init(sm.bar(kBarEmpty + s), C::EMPTY_ARRIVALS);
+        }
+        for (int i = 0; i < kF8Ring; ++i) {
+            ptx::mbar_init(sm.bar(kBarF8Full + i), 1);
+            ptx::mbar_init(sm.bar(kBarF8Empty + i), 4);
+        }
+        for (int i = 0; i < kScBufs; ++i) {
+            ptx::mbar_init(sm.bar(kBarScFull + i), 4);   // the four converter warps
+            ptx::mbar_init(sm.bar(kBarScEmpty + i), 4);  // the four softmax warps
         }
         ptx::mbar_init(sm.bar(kBarQFull), 1);
         ptx::mbar_init(sm.bar(kBarQEmpty), 1);
@@ -1057,6 +1238,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
         ptx::fence_mbar_init();
         ptx::tma_prefetch_map(kv_map);
         ptx::tma_prefetch_map(q_map);
+        if (F8) ptx::tma_prefetch_map(sc_map);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(sm.tmem_holder), C::TMEM_COLS);
@@ -1101,23 +1283,23 @@ __device__ __forceinline__ void decode_teardown(uint32_t tmem)
 
 // Warps: 0 producer, 1 score MMA (and TMEM owner), 2-5 softmax + epilogue,
 // 6-9 transposer, 10 output MMA.
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
-                  const DecodeParams p)
+                  const __grid_constant__ CUtensorMap sc_map, const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     Smem sm;
     Range w;
     uint32_t tmem;
     ptx::griddep_launch_dependents();
-    if (decode_setup<N, SQ>(p, &kv_map, &q_map, smem_raw, sm, w, tmem)) {
+    if (decode_setup<N, SQ, F8>(p, &kv_map, &q_map, &sc_map, smem_raw, sm, w, tmem)) {
         const int warp = threadIdx.x >> 5;
         const int g = blockIdx.x % p.G;
-        if (warp == 0) producer_warp<N, SQ>(p, w, g, sm, &kv_map, &q_map);
+        if (warp == 0) producer_warp<N, SQ, F8>(p, w, g, sm, &kv_map, &q_map, &sc_map);
         else if (warp == 1) score_mma_warp<N, SQ>(p, w, sm, tmem);
-        else if (warp < 6) softmax_warps<N, SQ>(p, w, g, sm, tmem);
-        else if (warp < 10) transposer_warps<N, SQ>(p, w, sm, tmem);
+        else if (warp < 6) softmax_warps<N, SQ, F8>(p, w, g, sm, tmem);
+        else if (warp < 10) transposer_warps<N, SQ, F8>(p, w, sm, tmem);
         else output_mma_warp<N, SQ>(p, w, sm, tmem);
     }
     decode_teardown<N, SQ>(tmem);
@@ -1297,9 +1479,10 @@ struct DeviceInfo {
 std::mutex g_dev_mutex;
 DeviceInfo g_dev[64];
 
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 int kernel_index()
 {
+    if (F8) return 7;
     if (N == 16 && SQ == 1) return 0;
     if (N == 32 && SQ == 1) return 1;
     if (N == 32 && SQ == 2) return 2;
@@ -1309,20 +1492,21 @@ int kernel_index()
     return 6;
 }
 
-template <int N, int SQ>
+template <int N, int SQ, bool F8>
 int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
-    const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024);
+    const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024 +
+                                       (F8 ? kF8Ring * kF8Unit + kScBytes : 0));
     int R = (smem_optin - fixed) / static_cast<int>(C::SLOT_BYTES);
     if (R > kMaxRing) R = kMaxRing;
     *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * C::SLOT_BYTES;
     return R;
 }
 
-template <int N, int SQ>
-mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, DecodeParams prm, int grid,
-                           cudaStream_t stream)
+template <int N, int SQ, bool F8>
+mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, const CUtensorMap &sc_map,
+                           DecodeParams prm, int grid, cudaStream_t stream)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1346,13 +1530,14 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
         return MLA_ERR_CUDA;
     }
     size_t smem = 0;
-    const int R = ring_for<N, SQ>(info.smem_optin, &smem);
+    const int R = ring_for<N, SQ, F8>(info.smem_optin, &smem);
     if (R * Cfg<N, SQ>::CPS < kMinRingChunks) {
         snprintf(g_last_error, sizeof g_last_error, "not enough shared memory for a %d-chunk ring", kMinRingChunks);
         return MLA_ERR_CUDA;
     }
-    const int ki = kernel_index<N, SQ>();
-    void (*kernel)(const CUtensorMap, const CUtensorMap, const DecodeParams) = mla_decode_kernel<N, SQ>;
+    const int ki = kernel_index<N, SQ, F8>();
+    void (*kernel)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const DecodeParams) =
+        mla_decode_kernel<N, SQ, F8>;
     if (!info.attr_set[ki]) {
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -1373,7 +1558,7 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, kv_map, q_map, prm);
+    e = cudaLaunchKernelEx(&cfg, kernel, kv_map, q_map, sc_map, prm);
     if (e != cudaSuccess) return cuda_fail(e, "mla_decode_kernel launch");
     return MLA_OK;
 }
@@ -1411,6 +1596,40 @@ mla_status_t static_workspace_address(void **out)
     }
     *out = g_static_ws_ptr[dev];
     return MLA_OK;
+}
+
+DecodeParams make_params(const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
+                         const Shape &sh, int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                         const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                         const WorkspaceLayout &wl, uint16_t *out, float *lse)
+{
+    DecodeParams prm;
+    prm.block_table = block_table;
+    prm.seqlens = cache_seqlens;
+    prm.sched = sched_meta;
+    prm.split_base = num_splits;
+    prm.ws_o = static_cast<float *>(workspace);
+    prm.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + wl.lse_off);
+    prm.out = out;
+    prm.lse = lse;
+    prm.err = const_cast<int32_t *>(sched_meta);
+    prm.B = B;
+    prm.s_q = s_q;
+    prm.H = H;
+    prm.G = sh.G;
+    prm.num_sms = num_sms;
+    prm.num_tuples = num_sms / sh.G;
+    prm.max_blocks = max_blocks;
+    prm.num_blocks = num_blocks;
+    prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+    prm.ring = 0;
+    prm.max_pieces = wl.pieces;
+    // Test hook (failure detection): MLA_DEBUG_STALL_CTA=k makes CTA k wait
+    // for a load that is never issued; its waits run out after their time
+    // limit and set MLA_DEVERR_TIMEOUT.  Unset in normal use.
+    prm.debug_stall_cta = -1;
+    if (const char *e = getenv("MLA_DEBUG_STALL_CTA")) prm.debug_stall_cta = atoi(e);
+    return prm;
 }
 
 }  // namespace host
@@ -1548,43 +1767,20 @@ mla_status_t mla_decode_attention(const uint16_t *q, const uint16_t *kv_cache, c
         }
     }
 
-    DecodeParams prm;
-    prm.block_table = block_table;
-    prm.seqlens = cache_seqlens;
-    prm.sched = sched_meta;
-    prm.split_base = num_splits;
-    prm.ws_o = static_cast<float *>(workspace);
-    prm.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + wl.lse_off);
-    prm.out = out;
-    prm.lse = lse;
-    prm.err = const_cast<int32_t *>(sched_meta);
-    prm.B = B;
-    prm.s_q = s_q;
-    prm.H = H;
-    prm.G = sh.G;
-    prm.num_sms = num_sms;
-    prm.num_tuples = num_sms / sh.G;
-    prm.max_blocks = max_blocks;
-    prm.num_blocks = num_blocks;
-    prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-    prm.ring = 0;
-    prm.max_pieces = wl.pieces;
-    // Test hook (failure detection): MLA_DEBUG_STALL_CTA=k makes CTA k wait
-    // for a load that is never issued; its waits run out after their time
-    // limit and set MLA_DEVERR_TIMEOUT.  Unset in normal use.
-    prm.debug_stall_cta = -1;
-    if (const char *e = getenv("MLA_DEBUG_STALL_CTA")) prm.debug_stall_cta = atoi(e);
+    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
+                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
     const int grid = prm.num_tuples * sh.G;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     mla_status_t rc;
-    if (sh.N == 16) rc = launch_decode<16, 1>(kv_map, q_map, prm, grid, st);
-    else if (sh.N == 32 && s_q == 1) rc = launch_decode<32, 1>(kv_map, q_map, prm, grid, st);
-    else if (sh.N == 32) rc = launch_decode<32, 2>(kv_map, q_map, prm, grid, st);
-    else if (s_q == 1) rc = launch_decode<64, 1>(kv_map, q_map, prm, grid, st);
-    else if (s_q == 2) rc = launch_decode<64, 2>(kv_map, q_map, prm, grid, st);
-    else if (s_q == 4) rc = launch_decode<64, 4>(kv_map, q_map, prm, grid, st);
-    else rc = launch_decode<64, 8>(kv_map, q_map, prm, grid, st);
+    // (the scale map is only read by the FP8 kernel; q_map stands in for it)
+    if (sh.N == 16) rc = launch_decode<16, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (sh.N == 32 && s_q == 1) rc = launch_decode<32, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (sh.N == 32) rc = launch_decode<32, 2, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 1) rc = launch_decode<64, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 2) rc = launch_decode<64, 2, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 4) rc = launch_decode<64, 4, false>(kv_map, q_map, q_map, prm, grid, st);
+    else rc = launch_decode<64, 8, false>(kv_map, q_map, q_map, prm, grid, st);
     return rc;
 }
 
@@ -1597,6 +1793,101 @@ mla_status_t mla_decode(const uint16_t *q, const uint16_t *kv_cache, const int32
         mla_decode_attention(q, kv_cache, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks,
                              softmax_scale, num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse,
                              stream);
+    if (rc != MLA_OK) return rc;
+    return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
+                              stream);
+}
+
+mla_status_t mla_decode_attention_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                                      const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q,
+                                      int H, int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                                      const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                                      size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
+{
+    if (!q || !kv_codes || !kv_scale || !block_table || !cache_seqlens || !sched_meta || !num_splits ||
+        !workspace || !out || !lse)
+        return MLA_ERR_INVALID_ARG;
+    if (B < 1 || B > kMaxBatch || num_blocks < 1 || num_blocks > INT32_MAX || max_blocks < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    Shape sh;
+    if (!resolve(s_q, H, &sh) || sh.N != 16 || s_q != 1) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (num_sms < sh.G || num_sms > kMaxSms) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 15) ||
+        (reinterpret_cast<uintptr_t>(kv_scale) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+        (reinterpret_cast<uintptr_t>(out) & 7) || (reinterpret_cast<uintptr_t>(lse) & 3) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3) ||
+        (reinterpret_cast<uintptr_t>(sched_meta) & 3) || (reinterpret_cast<uintptr_t>(num_splits) & 3))
+        return MLA_ERR_MISALIGNED;
+    const WorkspaceLayout wl = layout(B, s_q, sh, num_sms);
+    if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+
+    EncodeTiledFn encode = encode_fn();
+    if (!encode) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return MLA_ERR_CUDA;
+    }
+    CUtensorMap kv_map, q_map, sc_map;
+    // codes viewed as [num_blocks][64 rows][576 bytes]; box 128 bytes x 64 rows x 1 block, 128-byte
+    // swizzled.  The rope group's box (columns 512..639) reads zeros past column 575.
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage),
+                                    static_cast<cuuint64_t>(num_blocks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage) * kDQK};
+        const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(kPage), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        const CUresult r = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(kv_codes), dims,
+                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(kv fp8) failed: %d", static_cast<int>(r));
+            return MLA_ERR_CUDA;
+        }
+    }
+    // token scales viewed as [num_blocks][64]; box 64 x 1 block (256 bytes)
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kPage), static_cast<cuuint64_t>(num_blocks)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kPage) * 4};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kPage), 1};
+        const cuuint32_t estr[2] = {1, 1};
+        const CUresult r = encode(&sc_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(kv_scale), dims,
+                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(kv scale) failed: %d",
+                     static_cast<int>(r));
+            return MLA_ERR_CUDA;
+        }
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(B) * s_q * H};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDQK) * 2};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sh.HG)};
+        const cuuint32_t estr[2] = {1, 1};
+        const CUresult r = encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(q), dims,
+                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(q) failed: %d", static_cast<int>(r));
+            return MLA_ERR_CUDA;
+        }
+    }
+    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
+                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
+    return launch_decode<16, 1, true>(kv_map, q_map, sc_map, prm, prm.num_tuples * sh.G,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+mla_status_t mla_decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                            const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
+                            int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                            const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                            size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
+{
+    const mla_status_t rc =
+        mla_decode_attention_fp8(q, kv_codes, kv_scale, block_table, cache_seqlens, B, s_q, H, num_blocks,
+                                 max_blocks, softmax_scale, num_sms, sched_meta, num_splits, workspace,
+                                 workspace_bytes, out, lse, stream);
     if (rc != MLA_OK) return rc;
     return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
                               stream);

@@ -192,6 +192,33 @@ mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_c
                                          const int32_t *sched_meta, const int32_t *num_splits,
                                          uint16_t *out, float *lse, void *stream);
 
+/* FP8 cache.  The same decode over a cache of e4m3 codes with one fp32 scale
+ * per cached token: token j's row is e4m3(kv_codes[blk][j % 64][:]) *
+ * kv_scale[blk][j % 64] (the juejin.cn "FlashMLA" post, section 5, says
+ * FlashMLA runs in mixed precision such as FP8 and BF16; it fixes no format,
+ * and this per-token-scale layout is the reading taken).  Each tile's codes
+ * are widened in shared memory to bf16 (exactly: every e4m3 value is a bf16
+ * value) for the tensor-core MMAs; each token's scale multiplies its scores
+ * and its softmax weights in fp32, so the queries, the softmax and the
+ * outputs are as in mla_decode.
+ *   kv_codes   device uint8 [num_blocks, 64, 576] (e4m3 bit patterns, OCP E4M3
+ *              as __nv_fp8_e4m3 holds them), 16-byte aligned.
+ *   kv_scale   device fp32 [num_blocks, 64], 16-byte aligned.
+ *   Every other argument as for mla_decode (same metadata, same workspace).
+ * Supported shapes: s_q = 1 and H = 16 (16 query columns per CTA); others
+ * return MLA_ERR_UNSUPPORTED_SHAPE.  mla_decode_attention_fp8 launches the
+ * attention kernel alone, mla_decode_fp8 the attention and combine kernels. */
+mla_status_t mla_decode_attention_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                                      const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q,
+                                      int H, int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                                      const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                                      size_t workspace_bytes, uint16_t *out, float *lse, void *stream);
+mla_status_t mla_decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                            const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
+                            int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                            const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                            size_t workspace_bytes, uint16_t *out, float *lse, void *stream);
+
 /* Merge of W partial attention states of the same output rows, each computed
  * over a disjoint range of the tokens -- in context-parallel decode, the
  * (out, lse) of W ranks that each hold a contiguous range of every sequence's

@@ -110,3 +110,18 @@ def test_merge_states_rejects_bad_arguments(lib):
         bad = list(args)
         bad[i] = v
         assert lib.mla_merge_states(*bad) == status, (i, v)
+
+
+def test_decode_fp8_rejects_bad_arguments(lib):
+    def args(**kw):
+        a = dict(q=GOOD, codes=GOOD, scale=GOOD, bt=GOOD, sl=GOOD, B=8, s_q=1, H=16, nb=1024, mb=1024, sms=148)
+        a.update(kw)
+        return [P(a["q"]), P(a["codes"]), P(a["scale"]), P(a["bt"]), P(a["sl"]), a["B"], a["s_q"], a["H"],
+                a["nb"], a["mb"], ctypes.c_float(0.07), a["sms"], P(GOOD), P(GOOD), P(GOOD), 1 << 30,
+                P(GOOD), P(GOOD), P(0)]
+    assert lib.mla_decode_fp8(*args(codes=0)) == 1
+    assert lib.mla_decode_fp8(*args(scale=0)) == 1
+    assert lib.mla_decode_fp8(*args(H=32)) == 3      # 16 query columns only
+    assert lib.mla_decode_fp8(*args(s_q=2, H=8)) == 3
+    assert lib.mla_decode_fp8(*args(codes=GOOD + 8)) == 2
+    assert lib.mla_decode_fp8(*args(scale=GOOD + 4)) == 2

@@ -1,0 +1,85 @@
+"""FP8 (e4m3, one fp32 scale per cached token) cache on the GPU against the
+oracle's FP8 definition, through the C ABI (``mla_decode_fp8``)."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_latent_b200 as mla
+import mla_inputs as mi
+import oracle
+from test_parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    mla.load_library()
+    return torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+def run_fp8(inp, cache, dev, n_sms=None):
+    q, bt, sl = inp.q.to(dev), inp.block_table.to(dev), inp.cache_seqlens.to(dev)
+    n = mla.num_sms(dev) if n_sms is None else n_sms
+    sched, splits = mla.decode_metadata(sl, 1, inp.H, n)
+    out, lse = mla.decode_fp8(q, cache.codes.to(dev), cache.scale.to(dev), bt, sl, inp.scale, sched_meta=sched,
+                              num_splits=splits, num_sms_=n)
+    err = mla.get_device_error(sched)
+    return out.float().cpu().numpy(), lse.cpu().numpy(), err
+
+
+@pytest.mark.parametrize("seqlens,n_sms,pow2", [
+    ([1, 200, 700], None, False), ([1, 200, 700], 8, True), ([64, 65, 127, 128, 129], 17, False),
+    ([64 * 40 + 3, 5000], None, False), ([0, 300, 0], 7, False),
+])
+def test_fp8_matches_oracle(dev, orc, seqlens, n_sms, pow2):
+    inp = mi.small(B=len(seqlens), s_q=1, H=16, seqlens=seqlens, seed=60)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=61, pow2_scales=pow2)
+    g_out, g_lse, err = run_fp8(inp, cache, dev, n_sms)
+    assert err == 0
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"fp8 {seqlens}")
+
+
+def test_fp8_tail_codes_never_reach_the_result(dev, orc):
+    # rows past a sequence's end hold NaN codes (0x7F) and a NaN scale
+    inp = mi.small(B=2, s_q=1, H=16, seqlens=[70, 130], seed=62)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=63)
+    for b, L in enumerate(inp.cache_seqlens.tolist()):
+        last = int(inp.block_table[b, (L - 1) // 64])
+        cache.codes[last, L % 64 or 64:, :] = 0x7F
+        cache.scale[last, L % 64 or 64:] = float("nan")
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err == 0 and np.all(np.isfinite(g_out)) and np.all(np.isfinite(g_lse))
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what="fp8 NaN tails")
+
+
+def test_fp8_paging_invariance(dev):
+    # the same logical rows through an identity and a shuffled table: bitwise equal
+    a = mi.small(B=2, s_q=1, H=16, seqlens=[300, 900], table="identity", seed=64)
+    b = mi.small(B=2, s_q=1, H=16, seqlens=[300, 900], table="shuffled", seed=64)
+    ca = mi.fp8_cache(a.kv_cache.shape[0], seed=65)
+    cb = mi.Fp8Cache(codes=torch.empty_like(ca.codes), scale=torch.empty_like(ca.scale))
+    for s in range(2):
+        for p in range((int(a.cache_seqlens[s]) + 63) // 64):
+            cb.codes[int(b.block_table[s, p])] = ca.codes[int(a.block_table[s, p])]
+            cb.scale[int(b.block_table[s, p])] = ca.scale[int(a.block_table[s, p])]
+    oa = run_fp8(a, ca, dev, 8)
+    ob = run_fp8(b, cb, dev, 8)
+    assert np.array_equal(oa[0], ob[0]) and np.array_equal(oa[1], ob[1])
+
+
+def test_fp8_unsupported_shape_is_refused(dev):
+    inp = mi.small(B=1, s_q=1, H=32, seqlens=[100], seed=66)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=67)
+    with pytest.raises(mla.MLAError):
+        mla.decode_fp8(inp.q.to(dev), cache.codes.to(dev), cache.scale.to(dev), inp.block_table.to(dev),
+                       inp.cache_seqlens.to(dev), inp.scale)
