@@ -30,7 +30,9 @@
  *                           launches it; exported for tests and timing);
  *     mla_merge_states      context-parallel decode: merges the results of
  *                           W ranks that each attended over their own range
- *                           of every sequence's pages.
+ *                           of every sequence's pages;
+ *     mla_decode_fp8        the decode over an FP8 (e4m3, per-token scale)
+ *                           cache (mla_decode_attention_fp8: attention only).
  *
  * Conventions for every call.
  *   - Pointers marked "device" are CUDA device pointers of the current
