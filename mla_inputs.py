@@ -211,3 +211,38 @@ def algorithmic_bytes(inp: Inputs) -> int:
 def algorithmic_flops(inp: Inputs) -> int:
     """2 * H * s_q * L * (576 + 512) summed over sequences."""
     return sum(2 * inp.H * inp.s_q * int(L) * (D_QK + D_V) for L in inp.cache_seqlens)
+
+
+# ------------------------------------------------- non-absorbed form inputs
+D_NOPE = 128   # decompressed key / value width per head
+D_ROPE = 64    # rope columns, the last 64 of a cached latent row
+
+
+@dataclass
+class NaiveInputs:
+    """Extra inputs of the non-absorbed form over the same latent cache: the
+    queries in the decompressed space and the per-head up-projections."""
+    q: torch.Tensor     # [B, s_q, H, 192] bf16: 128 key columns, then 64 rope
+    w_uk: torch.Tensor  # [H, 128, 512] bf16: row e of head h = latent coefficients of key dim e
+    w_uv: torch.Tensor  # [H, 128, 512] bf16: the same for value dim e
+
+
+def naive_inputs(B: int, s_q: int, H: int, seed: int = 0) -> NaiveInputs:
+    """Seeded queries and up-projection matrices (torch CPU generator, drawn in
+    the order q, w_uk, w_uv): q ~ N(0, 1); the matrices ~ N(0, 1/512), so a
+    decompressed key or value of an N(0, 1) latent row is again about N(0, 1).
+    Every value is drawn in fp32 and rounded to bf16."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, s_q, H, D_NOPE + D_ROPE, generator=g).to(torch.bfloat16)
+    w_uk = (torch.randn(H, D_NOPE, D_V, generator=g) / math.sqrt(D_V)).to(torch.bfloat16)
+    w_uv = (torch.randn(H, D_NOPE, D_V, generator=g) / math.sqrt(D_V)).to(torch.bfloat16)
+    return NaiveInputs(q=q, w_uk=w_uk, w_uv=w_uv)
+
+
+def naive_algorithmic_flops(inp: Inputs) -> int:
+    """FLOPs of the non-absorbed form per call: per visible token and head the
+    two up-projections (2 x 2 x 512 x 128), then the 192-wide score and the
+    128-wide value accumulation per query position."""
+    H, s_q = inp.H, inp.s_q
+    tokens = sum(int(L) for L in inp.cache_seqlens)
+    return tokens * H * (2 * 2 * D_V * D_NOPE + s_q * 2 * (D_NOPE + D_ROPE + D_NOPE))

@@ -70,6 +70,10 @@ class Oracle:
         self.lib.mla_oracle_direct_fp8.restype = ctypes.c_int
         self.lib.mla_oracle_merge_states.argtypes = [f64p, f64p, ctypes.c_int, ctypes.c_int64, f64p, f64p]
         self.lib.mla_oracle_merge_states.restype = ctypes.c_int
+        self.lib.mla_oracle_naive.argtypes = [u16p, u16p, u16p, u16p, i32p, i32p, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_double, i32p,
+                                               ctypes.c_int, f64p, f64p]
+        self.lib.mla_oracle_naive.restype = ctypes.c_int
         self.lib.mla_oracle_threads.argtypes = []
         self.lib.mla_oracle_threads.restype = ctypes.c_int
 
@@ -201,6 +205,32 @@ class Oracle:
             sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), B, s_q, H, codes.shape[0], bt.shape[1],
             float(scale), _f64(out), _f64(lse))
         self._check(rc, "mla_oracle_direct_fp8")
+        return out, lse
+
+    def naive(self, q, kv_cache, w_uk, w_uv, block_table, cache_seqlens, scale, seqs=None):
+        """The non-absorbed form: ``q`` bf16 [B, s_q, H, 192] (128 key columns,
+        then 64 rope), ``w_uk`` / ``w_uv`` bf16 [H, 128, 512].  Returns fp64 out
+        [B, s_q, H, 128] and lse [B, s_q, H]; rows of sequences not in ``seqs``
+        (when given) are left as NaN."""
+        qb = self._bits(q)
+        B, s_q, H, dq = qb.shape
+        assert dq == 192
+        kv = self._bits(kv_cache)
+        wk = self._bits(w_uk)
+        wv = self._bits(w_uv)
+        assert wk.shape == (H, 128, 512) and wv.shape == (H, 128, 512)
+        assert kv.ndim == 3 and kv.shape[1:] == (64, 576)
+        bt = self._i32(block_table)
+        sl = self._i32(cache_seqlens)
+        out = np.full((B, s_q, H, 128), np.nan)
+        lse = np.full((B, s_q, H), np.nan)
+        arr, ptr, n = self._seq_list(seqs)
+        u16 = ctypes.POINTER(ctypes.c_uint16)
+        rc = self.lib.mla_oracle_naive(
+            qb.ctypes.data_as(u16), kv.ctypes.data_as(u16), wk.ctypes.data_as(u16), wv.ctypes.data_as(u16),
+            bt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            B, s_q, H, kv.shape[0], bt.shape[1], float(scale), ptr, n, _f64(out), _f64(lse))
+        self._check(rc, "mla_oracle_naive")
         return out, lse
 
     def threads(self) -> int:

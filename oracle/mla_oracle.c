@@ -50,7 +50,12 @@
  *                           (the context-parallel form: each of W ranks
  *                           attends over its own range of the tokens);
  *   mla_oracle_direct_fp8   the definition over an FP8 (e4m3) cache with one
- *                           fp32 scale per cached token.
+ *                           fp32 scale per cached token;
+ *   mla_oracle_naive        the non-absorbed form: each token's key and value
+ *                           decompressed from its latent row by per-head
+ *                           up-projection matrices, then softmax(Q K^T) V
+ *                           with 192-wide keys and 128-wide values (see the
+ *                           comment above that function).
  * They agree to rounding; the tests pin each one to closed forms, library
  * routines and invariants.
  */
@@ -63,6 +68,8 @@
 #endif
 
 #define ORC_DQK 576   /* q / k row width: 512 latent + 64 rope           */
+#define ORC_DNOPE 128 /* non-absorbed form: decompressed key / value width */
+#define ORC_DROPE 64  /* rope columns (the last 64 of a cached row)        */
 #define ORC_DV 512    /* v width: the first 512 columns of the same row   */
 #define ORC_PAGE 64   /* tokens per paged block                          */
 
@@ -601,4 +608,109 @@ int mla_oracle_direct_fp8(const uint16_t *q, const uint8_t *kv_codes, const floa
         free(row); free(sc);
     }
     return failed == 2 ? ORC_BAD_BLOCK : failed ? ORC_NO_MEMORY : ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Non-absorbed form.  "FlashMLA: compressing the KV cache to one eighth"    */
+/* (jsqmd.com), "MLA compression principle" and "FlashMLA compute flow",     */
+/* steps 1-5: the cache holds a compressed latent row per token, and each    */
+/* KV tile is decompressed when it is used -- K_tile = C_KV_tile W_UK,       */
+/* V_tile = C_KV_tile W_UV -- before S = Q K^T, the online softmax and       */
+/* O += softmax(S) V.  With the latent rows of the absorbed form (512 latent */
+/* columns c, then 64 rope columns) and per-head matrices:                   */
+/*   k_j[e]        = sum_{c<512} C_j[c] * w_uk[h][e][c]     e < 128          */
+/*   k_j[128 + r]  = C_j[512 + r]                           r < 64 (rope)    */
+/*   v_j[e]        = sum_{c<512} C_j[c] * w_uv[h][e][c]     e < 128          */
+/*   s_j           = scale * sum_{d<192} q[b,i,h,d] * k_j[d]                 */
+/*   out[e]        = sum_j softmax(s)_j * v_j[e],  lse = ln sum_j exp(s_j)   */
+/* over the same visible tokens as the absorbed form.  Readings: the rope    */
+/* columns are cached already rotated and are shared by every head (the      */
+/* absorbed form's layout), so no rotation happens here; the up-projection   */
+/* matrices are stored as [H][128][512] (row e of head h holds the latent    */
+/* coefficients of output dimension e).  Everything in fp64, decompressed    */
+/* per token without any intermediate rounding.                              */
+/*   q     [B, s_q, H, 192] bf16 (128 decompressed-key columns, then rope)   */
+/*   w_uk, w_uv  [H, 128, 512] bf16                                          */
+/*   out   [B, s_q, H, 128], lse [B, s_q, H] (fp64)                          */
+/* ------------------------------------------------------------------------ */
+int mla_oracle_naive(const uint16_t *q, const uint16_t *kv_cache, const uint16_t *w_uk, const uint16_t *w_uv,
+                     const int32_t *block_table, const int32_t *seqlens,
+                     int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                     double scale, const int32_t *seq_list, int n_seq_list,
+                     double *out, double *lse)
+{
+    /* q is not a 576-wide row here: the page-table check only needs the
+     * cache, so the problem record carries the cache with a stand-in q */
+    problem_t p = {kv_cache, kv_cache, block_table, seqlens, B, s_q, H, num_blocks, max_blocks, scale};
+    if (!q || !w_uk || !w_uv) return ORC_BAD_ARG;
+    int rc = check_problem(&p);
+    if (rc != ORC_OK) return rc;
+    const int nb = list_len(&p, seq_list, n_seq_list);
+    const int64_t rows = (int64_t)nb * s_q * H;
+    const int dq = ORC_DNOPE + ORC_DROPE;
+    int failed = 0;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int b = list_at(seq_list, (int)(r / ((int64_t)s_q * H)));
+        const int i = (int)((r / H) % s_q);
+        const int h = (int)(r % H);
+        const int64_t n = visible_tokens(seqlens[b], s_q, i);
+        double *o = out + (((int64_t)b * s_q + i) * H + h) * ORC_DNOPE;
+        double *ls = lse + ((int64_t)b * s_q + i) * H + h;
+        for (int e = 0; e < ORC_DNOPE; ++e) o[e] = 0.0;
+        if (n == 0) {
+            *ls = -INFINITY;
+            continue;
+        }
+        double *s = (double *)malloc((size_t)n * sizeof(double));
+        double *v = (double *)malloc((size_t)n * ORC_DNOPE * sizeof(double));
+        double *wk = (double *)malloc((size_t)ORC_DNOPE * ORC_DV * sizeof(double));
+        double *wv = (double *)malloc((size_t)ORC_DNOPE * ORC_DV * sizeof(double));
+        if (!s || !v || !wk || !wv) {
+            failed = 1;
+            free(s); free(v); free(wk); free(wv);
+            continue;
+        }
+        const uint16_t *wkh = w_uk + (int64_t)h * ORC_DNOPE * ORC_DV;
+        const uint16_t *wvh = w_uv + (int64_t)h * ORC_DNOPE * ORC_DV;
+        for (int64_t t = 0; t < (int64_t)ORC_DNOPE * ORC_DV; ++t) {
+            wk[t] = bf16_to_double(wkh[t]);
+            wv[t] = bf16_to_double(wvh[t]);
+        }
+        double qv[ORC_DNOPE + ORC_DROPE];
+        const uint16_t *qr = q + (((int64_t)b * s_q + i) * H + h) * dq;
+        for (int d = 0; d < dq; ++d) qv[d] = bf16_to_double(qr[d]);
+
+        /* per token: decompress k and v from the latent row, score */
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            const uint16_t *row = token_row(&p, b, j);
+            double c[ORC_DV];
+            for (int x = 0; x < ORC_DV; ++x) c[x] = bf16_to_double(row[x]);
+            double dot = 0.0;
+            for (int e = 0; e < ORC_DNOPE; ++e) {
+                double ke = 0.0, ve = 0.0;
+                for (int x = 0; x < ORC_DV; ++x) {
+                    ke += c[x] * wk[(int64_t)e * ORC_DV + x];
+                    ve += c[x] * wv[(int64_t)e * ORC_DV + x];
+                }
+                dot += qv[e] * ke;
+                v[j * ORC_DNOPE + e] = ve;
+            }
+            for (int x = 0; x < ORC_DROPE; ++x) dot += qv[ORC_DNOPE + x] * bf16_to_double(row[ORC_DV + x]);
+            s[j] = scale * dot;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            const double w = exp(s[j] - m);
+            l += w;
+            for (int e = 0; e < ORC_DNOPE; ++e) o[e] += w * v[j * ORC_DNOPE + e];
+        }
+        for (int e = 0; e < ORC_DNOPE; ++e) o[e] /= l;
+        *ls = m + log(l);
+        free(s); free(v); free(wk); free(wv);
+    }
+    return failed ? ORC_NO_MEMORY : ORC_OK;
 }

@@ -369,7 +369,91 @@ def pin_fp8_cache_against_sdpa(orc):
         _close(lse[b, 0], torch.logsumexp(s, dim=-1).numpy(), rel=1e-11, what="fp8 lse vs logsumexp")
 
 
+def _selection_matrix(H, perm_seed, rng_cols=512):
+    """[H, 128, 512] bf16 matrices whose row e of head h has a single 1, in a
+    seeded column: decompression then copies 128 chosen latent columns."""
+    g = torch.Generator().manual_seed(perm_seed)
+    w = torch.zeros(H, 128, rng_cols)
+    cols = []
+    for h in range(H):
+        c = torch.randperm(rng_cols, generator=g)[:128]
+        w[h, torch.arange(128), c] = 1.0
+        cols.append(c)
+    return w.to(torch.bfloat16), cols
+
+
+def pin_naive_selection_equals_absorbed(orc):
+    """Non-absorbed form with up-projections that select latent columns (k_e =
+    C[a_e], v_e = C[b_e]) against the absorbed form: absorbing the key matrix
+    into the query gives the 576-wide query q~[a_e] = q[e], q~[512 + r] =
+    q[128 + r] (exact in bf16), so the scores, hence lse, must agree to
+    rounding, and the output must be the absorbed output's columns b_e."""
+    lens = [1, 70, 129, 300]
+    base = mi.small(B=len(lens), s_q=2, H=3, seqlens=lens, seed=70)
+    nv = mi.naive_inputs(len(lens), 2, 3, seed=71)
+    w_uk, a_cols = _selection_matrix(3, 72)
+    w_uv, b_cols = _selection_matrix(3, 73)
+    out, lse = orc.naive(nv.q, base.kv_cache, w_uk, w_uv, base.block_table, base.cache_seqlens, base.scale)
+    qt = torch.zeros(len(lens), 2, 3, 576)
+    qf = nv.q.to(torch.float32)
+    for h in range(3):
+        qt[:, :, h, a_cols[h]] = qf[:, :, h, :128]
+        qt[:, :, h, 512:] = qf[:, :, h, 128:]
+    a_out, a_lse = orc.direct(qt.to(torch.bfloat16), base.kv_cache, base.block_table, base.cache_seqlens,
+                              base.scale)
+    _close(lse, a_lse, what="naive lse vs absorbed")
+    for h in range(3):
+        _close(out[:, :, h], a_out[:, :, h][..., b_cols[h].numpy()], what=f"naive out vs absorbed h={h}")
+
+
+def pin_naive_against_sdpa(orc):
+    """Dense random up-projections: keys and values decompressed with torch
+    float64 matmuls, then torch's scaled_dot_product_attention and logsumexp;
+    ragged lengths, s_q = 2 (query i sees seqlen - 1 + i tokens)."""
+    lens = [1, 2, 64, 65, 200]
+    base = mi.small(B=len(lens), s_q=2, H=2, seqlens=lens, seed=74)
+    nv = mi.naive_inputs(len(lens), 2, 2, seed=75)
+    out, lse = orc.naive(nv.q, base.kv_cache, nv.w_uk, nv.w_uv, base.block_table, base.cache_seqlens, base.scale)
+    q = torch.from_numpy(_bf16_to_f64(nv.q))
+    wk = torch.from_numpy(_bf16_to_f64(nv.w_uk))
+    wv = torch.from_numpy(_bf16_to_f64(nv.w_uv))
+    for b, L in enumerate(lens):
+        rows = torch.from_numpy(_rows_of(base, b, L))
+        for i in range(2):
+            n = max(0, L - 1 + i)
+            if n == 0:
+                assert np.all(out[b, i] == 0) and np.all(np.isneginf(lse[b, i])), "empty context"
+                continue
+            for h in range(2):
+                k = torch.cat([rows[:n, :512] @ wk[h].T, rows[:n, 512:]], dim=1)   # [n, 192]
+                v = rows[:n, :512] @ wv[h].T                                       # [n, 128]
+                qq = q[b, i, h].view(1, 1, 192)
+                ref = torch.nn.functional.scaled_dot_product_attention(qq, k.unsqueeze(0), v.unsqueeze(0),
+                                                                       scale=base.scale)
+                _close(out[b, i, h], ref[0, 0].numpy(), what=f"naive sdpa b={b} i={i} h={h}")
+                _close(lse[b, i, h], torch.logsumexp(base.scale * (k @ q[b, i, h]), dim=0).numpy(),
+                       what=f"naive lse b={b} i={i} h={h}")
+
+
+def pin_naive_single_token(orc):
+    """A one-token context returns that token's decompressed value exactly
+    (numpy matmul of the latent row with the value matrix) and lse = the
+    scaled score of its decompressed key."""
+    base = mi.small(B=2, s_q=1, H=2, seqlens=[1, 1], seed=76)
+    nv = mi.naive_inputs(2, 1, 2, seed=77)
+    out, lse = orc.naive(nv.q, base.kv_cache, nv.w_uk, nv.w_uv, base.block_table, base.cache_seqlens, base.scale)
+    q = _bf16_to_f64(nv.q)
+    wk, wv = _bf16_to_f64(nv.w_uk), _bf16_to_f64(nv.w_uv)
+    for b in range(2):
+        row = _rows_of(base, b, 1)[0]
+        for h in range(2):
+            _close(out[b, 0, h], wv[h] @ row[:512], what="single-token value")
+            key = np.concatenate([wk[h] @ row[:512], row[512:]])
+            _close(lse[b, 0, h], base.scale * float(q[b, 0, h] @ key), what="single-token lse")
+
+
 ALL_PINS = [
+    pin_naive_selection_equals_absorbed, pin_naive_against_sdpa, pin_naive_single_token,
     pin_single_token,
     pin_equal_scores_mean_of_values,
     pin_zero_scale,

@@ -12,9 +12,11 @@ from oracle_pins import ALL_PINS
 
 # (description, text in mla_oracle.c, replacement); each text must occur once.
 MUTANTS = [
-    ("dropped softmax scale", "s[j] = scale * dot;", "s[j] = dot;"),
-    ("wrong sign in the exponent", "const double w = exp(s[j] - m);\n            l += w;",
-     "const double w = exp(m - s[j]);\n            l += w;"),
+    ("dropped softmax scale", "dot += qv[d] * bf16_to_double(k[d]);\n            s[j] = scale * dot;",
+     "dot += qv[d] * bf16_to_double(k[d]);\n            s[j] = dot;"),
+    ("wrong sign in the exponent",
+     "const uint16_t *k = token_row(&p, b, j);\n            const double w = exp(s[j] - m);",
+     "const uint16_t *k = token_row(&p, b, j);\n            const double w = exp(m - s[j]);"),
     ("value read from the wrong columns", "o[c] += w * bf16_to_double(k[c]);",
      "o[c] += w * bf16_to_double(k[c + 64]);"),
     ("causal window off by one", "int64_t n = seqlen - s_q + 1 + i;", "int64_t n = seqlen - s_q + i;"),
@@ -43,6 +45,14 @@ MUTANTS = [
      "if (ex == 0) mag = ldexp((double)mant, -10);"),
     ("fp8 token scale dropped", "row[j * ORC_DQK + d] = table[kv_codes[tok * ORC_DQK + d]] * ks;",
      "row[j * ORC_DQK + d] = table[kv_codes[tok * ORC_DQK + d]];"),
+    ("non-absorbed: key matrix read transposed", "ke += c[x] * wk[(int64_t)e * ORC_DV + x];",
+     "ke += c[x] * wk[(int64_t)x * ORC_DNOPE + e];"),
+    ("non-absorbed: value decompressed with the key matrix", "ve += c[x] * wv[(int64_t)e * ORC_DV + x];",
+     "ve += c[x] * wk[(int64_t)e * ORC_DV + x];"),
+    ("non-absorbed: rope part of the score dropped",
+     "for (int x = 0; x < ORC_DROPE; ++x) dot += qv[ORC_DNOPE + x] * bf16_to_double(row[ORC_DV + x]);", ""),
+    ("non-absorbed: head of the up-projections ignored",
+     "const uint16_t *wkh = w_uk + (int64_t)h * ORC_DNOPE * ORC_DV;", "const uint16_t *wkh = w_uk;"),
 ]
 
 
