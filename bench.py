@@ -11,11 +11,12 @@ The inputs are larger than the 126 MB L2 and consecutive steps read two
 different device copies of the cache, so no step can find the cache in L2.
 
 Printed (rank 0, one JSON line): metric / value / unit (microseconds per call,
-lower is better), the attention kernel's roofline against the measured HBM
-copy bandwidth, an end-to-end figure through the same C ABI with the step's
-inputs copied from pinned host memory and its outputs copied back inside the
-timed region, the SM clocks sampled during the timed region, and the fp64
-CPU oracle timed on a bounded sample as a baseline.
+lower is better), the kernel's roofline against the measured HBM copy
+bandwidth, the error against the fp64 oracle on sampled sequences, an
+end-to-end figure through the same C ABI with the step's inputs copied from
+pinned host memory and its outputs copied back inside the timed region, the
+SM clocks sampled during the timed region, and the fp64 CPU oracle timed on a
+bounded sample as a baseline.
 
 With N > 1 (launched by torchrun) every rank runs its own replica of the
 workload on its own GPU (independent batches, no collective on the data
@@ -249,12 +250,24 @@ def cpu_baseline(inp: mi.Inputs, target_s: float = 15.0):
                       f"{inp.s_q * inp.H} query rows each, {t:.2f} s, scaled by {work_full / work_sample:.1f}"}
 
 
+def selected_workload(args) -> mi.Workload:
+    """The workload named on the command line, with its batch cut to
+    ``--batch`` sequences when given (a smaller case of the same shape and
+    length distribution, for profiler captures that must stay small)."""
+    w = mi.WORKLOADS[args.workload]
+    if args.batch:
+        if not 1 <= args.batch <= w.B:
+            raise SystemExit(f"--batch must be in [1, {w.B}] for {w.name}")
+        w = mi.workload(args.workload, B=args.batch)
+    return w
+
+
 def run_reference(args, world, rank):
     """The CPU oracle as the reference arm (rank 0 only)."""
     if rank != 0:
         return 0
     import oracle
-    w = mi.WORKLOADS[args.workload]
+    w = selected_workload(args)
     inp = mi.make_inputs(w, seed=0)
     orc = oracle.default()
     full_tokens = int(inp.cache_seqlens.max())
@@ -285,6 +298,37 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------- GPU arm
+# sequences the oracle recomputes for the accuracy figures of each workload
+ACCURACY_SAMPLE = {
+    "b1_h16_l1k_identity": None,
+    "b16_h16_l4k": None,
+    "b32_sq2_h16_l16k_outliers": [0, 13, 31],
+    "b64_h128_lvar1k32k": [0, 7, 33, 63],
+    "b8_h16_l64k": [0, 5],
+}
+
+
+def accuracy(g_out, g_lse, r_out, r_lse, seqs, B):
+    """Error of the GPU result against the fp64 oracle on sampled sequences:
+    max |out err|, relative RMSE sqrt(sum err^2 / sum ref^2) over those
+    outputs, and max |lse err| (the figures and bounds the tests assert)."""
+    import numpy as np
+    if seqs is not None:
+        g_out, g_lse, r_out, r_lse = g_out[seqs], g_lse[seqs], r_out[seqs], r_lse[seqs]
+    err = np.abs(g_out.astype(np.float64) - r_out)
+    den = float(np.sum(r_out ** 2))
+    fin = np.isfinite(r_lse)
+    lerr = float(np.abs(g_lse[fin] - r_lse[fin]).max()) if fin.any() else 0.0
+    rmse = (float(np.sum(err ** 2)) / den) ** 0.5 if den > 0 else 0.0
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(r_out), 1e-30))) - 7)
+    bound = np.where(np.abs(r_out) < 1.0, 1.5e-2, 1.5e-2 + ulp)
+    return {"sequences": "all" if seqs is None else f"{len(seqs)} of {B}: {seqs}",
+            "out_max_abs_err": float(err.max()), "out_rel_rmse": rmse, "lse_max_abs_err": lerr,
+            "out_max_abs_ref": float(np.abs(r_out).max()),
+            "within_bounds": bool(np.all(err <= bound) and rmse <= 5e-3 and lerr <= 1e-3),
+            "bounds": "out: 1.5e-2 where |ref| < 1, else 1.5e-2 + one bf16 ulp; rel RMSE 5e-3; lse 1e-3"}
+
+
 def run_ours(args, world, rank, local):
     import ctypes
 
@@ -294,7 +338,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     init_dist(world, "nccl")
     lib = mla.load_library()
-    w = mi.WORKLOADS[args.workload]
+    w = selected_workload(args)
     inp = mi.make_inputs(w, seed=rank)
     B, s_q, H = w.B, w.s_q, w.H
     n_sms = mla.num_sms(dev)
@@ -339,6 +383,17 @@ def run_ours(args, world, rank, local):
         call_metadata(); call_attention(kv_copies[k % n_copies]); call_combine()
     torch.cuda.synchronize(dev)
     assert mla.get_device_error(sched) == 0
+
+    # ---- accuracy against the fp64 oracle on sampled sequences (rank 0, N = 1)
+    acc = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        call_metadata(); call_attention(kv_copies[0]); call_combine()
+        torch.cuda.synchronize(dev)
+        seqs = ACCURACY_SAMPLE.get(args.workload) if not args.batch else [0]
+        r_out, r_lse = oracle.default().direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale,
+                                               seqs=seqs)
+        acc = accuracy(out.float().cpu().numpy(), lse.cpu().numpy(), r_out, r_lse, seqs, B)
 
     # ---- timed region 1: K steps, each on the other copy of the cache, with
     # an event between kernels to time each one
@@ -430,21 +485,6 @@ def run_ours(args, world, rank, local):
         graph_us = max_over_ranks(graph_us if graph_us is not None else float("nan"), dev)
     assert mla.get_device_error(sched) == 0
 
-    # ---- a read-only stream over 1 GiB in the same run (torch's sum), as a
-    # second bandwidth reference beside the copy figure
-    probe = torch.empty(1 << 28, dtype=torch.float32, device=dev).fill_(1.0)
-    best = None
-    for _ in range(5):
-        ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ra.record(stream)
-        probe.sum()
-        rb.record(stream)
-        torch.cuda.synchronize(dev)
-        t = ra.elapsed_time(rb)
-        best = t if best is None else min(best, t)
-    read_gbs = probe.numel() * 4 / (best * 1e-3) / 1e9
-    del probe
-
     # ---- end to end through the C ABI from pinned host memory: the step's
     # inputs (q, page table, lengths) sit back to back in one pinned buffer
     # and go over in one copy; out and lse come back in one copy.  The C ABI
@@ -488,10 +528,8 @@ def run_ours(args, world, rank, local):
     roof = roofline(alg_bytes, alg_flops, mean_attn_ms * 1e-3, measured_peaks())
     t_attn = mean_attn_ms * 1e-3
     roof["both"]["hbm_frac_of_nominal_8tbs"] = alg_bytes / t_attn / 8e12
-    roof["both"]["read_stream_gbs_measured_here"] = read_gbs
-    roof["both"]["hbm_frac_of_read_stream"] = alg_bytes / t_attn / (read_gbs * 1e9)
     roof["both"]["tensor_frac_of_sustained"] = alg_flops / t_attn / (sustained_tflops() * 1e12)
-    roof["traffic"] = ncu_traffic(args.workload)
+    roof["traffic"] = ncu_traffic(args.workload) if not args.batch else None
     roof["kernel"] = attention_kernel_name(s_q, H)
     roof["algorithmic_bytes_per_launch"] = alg_bytes
     roof["algorithmic_flops_per_launch"] = alg_flops
@@ -527,6 +565,8 @@ def run_ours(args, world, rank, local):
                    "built once (region 3); cuda_graph_us: whole steps replayed from a CUDA graph"),
         "clocks": clocks,
     }
+    if acc is not None:
+        line["accuracy"] = acc
     if world > 1:
         line["aggregate_calls_per_s"] = world / (mean_step_ms * 1e-3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -553,7 +593,7 @@ def run_context_parallel_rank(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     lib = mla.load_library()
-    w = mi.WORKLOADS[args.workload]
+    w = selected_workload(args)
     if w.s_q != 1:
         raise SystemExit("context-parallel decode takes s_q = 1 workloads")
     inp = mi.make_inputs(w, seed=0)
@@ -624,8 +664,10 @@ def run_context_parallel_rank(args):
 
 def run_fp8(args):
     """The decode over an FP8 (e4m3, one fp32 scale per token) cache of the same
-    workload, one GPU: metadata + attention + combine per call, and the
-    attention kernel alone; its roofline counts 576 + 4 bytes per cached token."""
+    workload, one GPU: per call the metadata, attention and combine kernels
+    (as the default line), the attention kernel alone and its roofline on
+    576 + 4 bytes per cached token, and the error against the oracle's FP8
+    definition."""
     import ctypes
 
     import decode_attention_latent_b200 as mla
@@ -633,12 +675,12 @@ def run_fp8(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     lib = mla.load_library()
-    w = mi.WORKLOADS[args.workload]
+    w = selected_workload(args)
     if w.s_q != 1 or w.H != 16:
         raise SystemExit("the FP8 cache path takes s_q = 1, H = 16 workloads")
     inp = mi.make_inputs(w, seed=0)
     nb = inp.kv_cache.shape[0]
-    del inp.kv_cache
+    inp.kv_cache = None  # the bf16 cache is not used here
     cache = mi.fp8_cache(nb, seed=1)
     B, H = w.B, w.H
     n_sms = mla.num_sms(dev)
@@ -660,38 +702,53 @@ def run_fp8(args):
         assert lib.mla_decode_metadata(P(sl.data_ptr()), B, 1, H, n_sms, P(sched.data_ptr()),
                                        P(splits.data_ptr()), sp) == 0
 
-    def attn(k):
+    def decode(k, fn):
         c, s_ = codes[k % n_copies], scales[k % n_copies]
-        assert lib.mla_decode_attention_fp8(P(q.data_ptr()), P(c.data_ptr()), P(s_.data_ptr()), P(bt.data_ptr()),
-                                            P(sl.data_ptr()), B, 1, H, nb, bt.shape[1], ctypes.c_float(inp.scale),
-                                            n_sms, P(sched.data_ptr()), P(splits.data_ptr()), P(ws.data_ptr()),
-                                            ws_bytes, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
+        assert fn(P(q.data_ptr()), P(c.data_ptr()), P(s_.data_ptr()), P(bt.data_ptr()),
+                  P(sl.data_ptr()), B, 1, H, nb, bt.shape[1], ctypes.c_float(inp.scale),
+                  n_sms, P(sched.data_ptr()), P(splits.data_ptr()), P(ws.data_ptr()),
+                  ws_bytes, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
 
-    def comb():
-        assert lib.mla_decode_combine(P(splits.data_ptr()), P(sched.data_ptr()), P(ws.data_ptr()), ws_bytes, B, 1, H,
-                                      n_sms, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
+    def call(k):
+        meta()
+        decode(k, lib.mla_decode_fp8)
 
     for k in range(max(3, args.warmup)):
-        meta(); attn(k); comb()
+        call(k)
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    acc = None
+    if not args.no_cpu_baseline:
+        import oracle
+        call(0)
+        torch.cuda.synchronize(dev)
+        r_out, r_lse = oracle.default().direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table,
+                                                   inp.cache_seqlens, inp.scale)
+        acc = accuracy(out.float().cpu().numpy(), lse.cpu().numpy(), r_out, r_lse, None, B)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for k in range(args.steps):
-        meta(); attn(k); comb()
-    e1.record()
-    torch.cuda.synchronize(dev)
-    call_us = e0.elapsed_time(e1) * 1e3 / args.steps
-    meta()
-    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for k in range(args.steps):
-        a_ev[k][0].record(); attn(k); a_ev[k][1].record()
+        ev[k][0].record(); call(k); ev[k][1].record()
     torch.cuda.synchronize(dev)
     assert mla.get_device_error(sched) == 0
-    attn_us = statistics.mean(a.elapsed_time(b) for a, b in a_ev) * 1e3
+    call_us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    meta()
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for k in range(args.steps):
+        ea[k][0].record(); decode(k, lib.mla_decode_attention_fp8); ea[k][1].record()
+    torch.cuda.synchronize(dev)
+    assert mla.get_device_error(sched) == 0
+    attn_us = statistics.mean(a.elapsed_time(b) for a, b in ea) * 1e3
     tokens = int(inp.cache_seqlens.sum())
     alg = tokens * (576 + 4) + q.numel() * 2 + out.numel() * 2 + lse.numel() * 4 + sum(
-        (int(L) + 63) // 64 for L in inp.cache_seqlens.tolist()) * 4
+        (int(L) + 63) // 64 for L in inp.cache_seqlens.tolist()) * 4 + B * 4
     hbm = measured_peaks()[0]
+    traffic = None
+    path = os.path.join(ROOT, "profiles", f"mla_decode_fp8_{args.workload}.md")
+    if os.path.exists(path) and not args.batch:
+        text = open(path).read()
+        m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        m_s = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+        if m_b and m_s and m_s.group(1) == source_digest():
+            traffic = float(m_b.group(1))
     line = {
         "metric": "MLA decode us/call over an FP8 (e4m3, per-token scale) cache", "value": call_us, "unit": "us/call",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
@@ -700,8 +757,11 @@ def run_fp8(args):
         "attention_us": attn_us,
         "roofline": {"bound": "hbm", "achieved": alg / (attn_us * 1e-6) / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": alg / (attn_us * 1e-6) / 1e9 / hbm, "algorithmic_bytes_per_launch": alg,
-                     "traffic": None},
+                     "traffic": traffic, "kernel": "mla_decode_kernel<16,1,true>"},
+        "gpu_launches": 3 * args.steps,
     }
+    if acc is not None:
+        line["accuracy"] = acc
     print(json.dumps(line))
     return 0
 
@@ -714,6 +774,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=mi.HEADLINE, choices=sorted(mi.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="cut the workload to its first BATCH sequences (profiler captures on a smaller case)")
     ap.add_argument("--fp8", action="store_true", help="the same workload over an FP8 (e4m3) cache (H = 16, s_q = 1)")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="W",
                     help="time one rank of a W-way context-parallel decode on one GPU (s_q = 1 workloads)")

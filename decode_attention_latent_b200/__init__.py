@@ -42,7 +42,8 @@ EXPORTED = (
     "mla_sched_meta_ints", "mla_decode_workspace_size", "mla_decode_metadata",
     "mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_static_workspace",
     "mla_merge_states", "mla_decode_fp8", "mla_decode_attention_fp8", "mla_get_device_error",
-    "mla_status_string", "mla_last_error_message",
+    "mla_status_string", "mla_last_error_message", "mla_debug_stall_cta",
+    "mla_decode_naive", "mla_decode_naive_workspace_size",
 )
 
 
@@ -100,6 +101,13 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_last_error_message.argtypes = []
     lib.mla_last_error_message.restype = ctypes.c_char_p
+    lib.mla_debug_stall_cta.argtypes = [ci]
+    lib.mla_debug_stall_cta.restype = None
+    lib.mla_decode_naive_workspace_size.argtypes = [ci, ci, ci, ci, ci]
+    lib.mla_decode_naive_workspace_size.restype = sz
+    lib.mla_decode_naive.argtypes = [cu16p, cu16p, cu16p, cu16p, i32p, i32p, ci, ci, ci, ctypes.c_int64, ci,
+                                     ctypes.c_float, ci, vp, sz, i32p, cu16p, vp, vp]
+    lib.mla_decode_naive.restype = ci
     if path == LIBRARY:
         _lib = lib
     return lib
@@ -107,9 +115,7 @@ def load_library(path: str = LIBRARY) -> ctypes.CDLL:
 
 def _check(rc: int, where: str):
     if rc != MLA_OK:
-        detail = ""
-        if rc == 5:
-            detail = load_library().mla_last_error_message().decode(errors="replace")
+        detail = load_library().mla_last_error_message().decode(errors="replace")
         raise MLAError(rc, where, detail)
 
 
@@ -176,10 +182,12 @@ def decode(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor, c
            workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
            lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
            combine: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Absorbed-form MLA decode (``mla_decode``): returns (out bf16 [B,s_q,H,512],
-    lse fp32 [B,s_q,H]).  Builds the schedule when ``sched_meta`` is None.
+    """Absorbed-form MLA decode (``mla_decode``: the attention kernel, then the
+    combine kernel): returns (out bf16 [B,s_q,H,512], lse fp32 [B,s_q,H]).
+    Builds the schedule with ``decode_metadata`` when ``sched_meta`` is None.
     With ``combine=False`` only the attention kernel runs
-    (``mla_decode_attention``); the caller then runs ``decode_combine``."""
+    (``mla_decode_attention``), leaving split sequences as pieces in
+    ``workspace``; the caller then runs ``decode_combine``."""
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("q must be a CUDA tensor")
@@ -282,6 +290,63 @@ def decode_fp8(q: torch.Tensor, kv_codes: torch.Tensor, kv_scale: torch.Tensor, 
     return out, lse
 
 
+D_NAIVE = 128  # decompressed key / value width of the non-absorbed form
+
+
+def decode_naive(q: torch.Tensor, kv_cache: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor,
+                 block_table: torch.Tensor, cache_seqlens: torch.Tensor, softmax_scale: float, *,
+                 num_sms_: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+                 error_word: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Non-absorbed form (``mla_decode_naive``): ``q`` bf16 [B, s_q, H, 192]
+    (128 key columns, then 64 rope), the latent cache of ``decode``, ``w_uk``
+    / ``w_uv`` bf16 [H, 128, 512].  Returns (out bf16 [B, s_q, H, 128], lse
+    fp32 [B, s_q, H], the device error word int32 [1])."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("q must be a CUDA tensor")
+    if q.dim() != 4 or q.shape[-1] != D_NAIVE + D_QK - D_V:
+        raise ValueError("q must be [B, s_q, H, 192]")
+    B, s_q, H, _ = q.shape
+    _require(q, "q", torch.bfloat16, dev)
+    if kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (PAGE, D_QK):
+        raise ValueError(f"kv_cache must be [num_blocks, {PAGE}, {D_QK}]")
+    _require(kv_cache, "kv_cache", torch.bfloat16, dev)
+    _require(w_uk, "w_uk", torch.bfloat16, dev, (H, D_NAIVE, D_V))
+    _require(w_uv, "w_uv", torch.bfloat16, dev, (H, D_NAIVE, D_V))
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_blocks]")
+    _require(block_table, "block_table", torch.int32, dev)
+    _require(cache_seqlens, "cache_seqlens", torch.int32, dev, (B,))
+    n = num_sms(dev) if num_sms_ is None else int(num_sms_)
+    lib = load_library()
+    ws_bytes = int(lib.mla_decode_naive_workspace_size(B, s_q, H, block_table.shape[1], n))
+    if ws_bytes == 0:
+        raise MLAError(3, "mla_decode_naive_workspace_size", f"B={B} s_q={s_q} H={H}")
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if error_word is None:
+        error_word = torch.zeros(1, dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty(B, s_q, H, D_NAIVE, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(B, s_q, H, dtype=torch.float32, device=dev)
+    _require(workspace, "workspace", torch.uint8, dev)
+    _require(error_word, "error_word", torch.int32, dev, (1,))
+    _require(out, "out", torch.bfloat16, dev, (B, s_q, H, D_NAIVE))
+    _require(lse, "lse", torch.float32, dev, (B, s_q, H))
+    rc = lib.mla_decode_naive(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(kv_cache.data_ptr()), ctypes.c_void_p(w_uk.data_ptr()),
+        ctypes.c_void_p(w_uv.data_ptr()), ctypes.c_void_p(block_table.data_ptr()),
+        ctypes.c_void_p(cache_seqlens.data_ptr()), B, s_q, H, kv_cache.shape[0], block_table.shape[1],
+        float(softmax_scale), n, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+        ctypes.c_void_p(error_word.data_ptr()), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+        _stream_handle(stream, dev))
+    _check(rc, "mla_decode_naive")
+    return out, lse, error_word
+
+
 def merge_states(out_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optional[torch.Tensor] = None,
                  lse: Optional[torch.Tensor] = None,
                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -309,6 +374,13 @@ def merge_states(out_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optio
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), _stream_handle(stream, dev))
     _check(rc, "mla_merge_states")
     return out, lse
+
+
+def debug_stall_cta(cta: int) -> None:
+    """Test hook (``mla_debug_stall_cta``): CTA ``cta`` of the next decode
+    launches never loads its first chunk, so its bounded waits run out; -1
+    turns it off."""
+    load_library().mla_debug_stall_cta(int(cta))
 
 
 def get_device_error(sched_meta: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -15,7 +15,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "mla_decode.cu"), os.path.join(HERE, "csrc", "mla_merge.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "mla_decode.cu"), os.path.join(HERE, "csrc", "mla_merge.cu"),
+           os.path.join(HERE, "csrc", "mla_naive.cu")]
 HEADERS = [os.path.join(HERE, "csrc", "sm100_ptx.cuh"), os.path.join(ROOT, "include", "mla_decode.h")]
 LIBRARY = os.path.join(HERE, "libmla_decode_b200.so")
 

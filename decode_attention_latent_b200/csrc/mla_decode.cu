@@ -45,6 +45,7 @@
 #include <cstring>
 #include <climits>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mla_decode.h"
@@ -1470,6 +1471,87 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Encoded tensor maps, cached by everything that goes into the encoding (the
+// tensor's address, shape, strides, box and layout options): a repeated call
+// on the same buffers reuses the map instead of encoding it again.  A map
+// holds only an address and a shape, so a cached one stays valid for any
+// buffer that is later placed at the same address with the same shape.
+struct MapKey {
+    int dtype, rank, swizzle, promo;
+    const void *ptr;
+    cuuint64_t dims[3], strides[2];
+    cuuint32_t box[3];
+};
+
+struct MapEntry {
+    bool used;
+    MapKey key;
+    CUtensorMap map;
+};
+
+constexpr int kMapCache = 32;
+std::mutex g_map_mutex;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+
+bool same_key(const MapKey &a, const MapKey &b)
+{
+    if (a.dtype != b.dtype || a.rank != b.rank || a.swizzle != b.swizzle || a.promo != b.promo || a.ptr != b.ptr)
+        return false;
+    for (int i = 0; i < a.rank; ++i)
+        if (a.dims[i] != b.dims[i] || a.box[i] != b.box[i]) return false;
+    for (int i = 0; i + 1 < a.rank; ++i)
+        if (a.strides[i] != b.strides[i]) return false;
+    return true;
+}
+
+// Tiled tensor map of `rank` <= 3 dimensions (element strides 1, no
+// interleave, zero fill); returns false with the message set on failure.
+bool tensor_map(CUtensorMap *out, const char *what, CUtensorMapDataType dtype, int rank, const void *ptr,
+                const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle swizzle,
+                CUtensorMapL2promotion promo)
+{
+    MapKey key;
+    memset(&key, 0, sizeof key);
+    key.dtype = static_cast<int>(dtype);
+    key.rank = rank;
+    key.swizzle = static_cast<int>(swizzle);
+    key.promo = static_cast<int>(promo);
+    key.ptr = ptr;
+    for (int i = 0; i < rank; ++i) {
+        key.dims[i] = dims[i];
+        key.box[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides[i];
+    {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        for (int i = 0; i < kMapCache; ++i)
+            if (g_maps[i].used && same_key(g_maps[i].key, key)) {
+                *out = g_maps[i].map;
+                return true;
+            }
+    }
+    EncodeTiledFn encode = encode_fn();
+    if (!encode) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return false;
+    }
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = encode(out, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(%s) failed: %d", what, static_cast<int>(r));
+        return false;
+    }
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    MapEntry &e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.used = true;
+    e.key = key;
+    e.map = *out;
+    return true;
+}
+
 struct DeviceInfo {
     int smem_optin = 0;
     int major = 0;
@@ -1598,6 +1680,9 @@ mla_status_t static_workspace_address(void **out)
     return MLA_OK;
 }
 
+// Test hook for the bounded device waits (mla_debug_stall_cta): -1 = off.
+std::atomic<int> g_debug_stall_cta{-1};
+
 DecodeParams make_params(const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
                          const Shape &sh, int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
                          const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
@@ -1624,11 +1709,7 @@ DecodeParams make_params(const int32_t *block_table, const int32_t *cache_seqlen
     prm.scale_log2 = softmax_scale * 1.4426950408889634f;
     prm.ring = 0;
     prm.max_pieces = wl.pieces;
-    // Test hook (failure detection): MLA_DEBUG_STALL_CTA=k makes CTA k wait
-    // for a load that is never issued; its waits run out after their time
-    // limit and set MLA_DEVERR_TIMEOUT.  Unset in normal use.
-    prm.debug_stall_cta = -1;
-    if (const char *e = getenv("MLA_DEBUG_STALL_CTA")) prm.debug_stall_cta = atoi(e);
+    prm.debug_stall_cta = g_debug_stall_cta.load(std::memory_order_relaxed);
     return prm;
 }
 
@@ -1637,6 +1718,146 @@ DecodeParams make_params(const int32_t *block_table, const int32_t *cache_seqlen
 
 using namespace mla;
 using namespace mla::host;
+
+extern "C" mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_meta,
+                                          const void *workspace, size_t workspace_bytes, int B, int s_q, int H,
+                                          int num_sms, uint16_t *out, float *lse, void *stream);
+
+namespace mla {
+namespace host {
+
+void clear_error() { g_last_error[0] = '\0'; }
+
+// Checks shared by every decode entry point; `kv_align` is the cache
+// pointer's alignment rule.
+mla_status_t check_decode_args(const void *q, const void *kv, const void *kv_scale, bool fp8,
+                               const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
+                               int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                               const int32_t *sched_meta, const int32_t *num_splits, const void *workspace,
+                               size_t workspace_bytes, const uint16_t *out, const float *lse, Shape *sh,
+                               WorkspaceLayout *wl)
+{
+    if (!q || !kv || (fp8 && !kv_scale) || !block_table || !cache_seqlens || !sched_meta || !num_splits ||
+        !workspace || !out || !lse)
+        return MLA_ERR_INVALID_ARG;
+    if (B < 1 || B > kMaxBatch || num_blocks < 1 || num_blocks > INT32_MAX || max_blocks < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    if (!resolve(s_q, H, sh)) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (fp8 && (sh->N != 16 || s_q != 1)) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (num_sms < sh->G || num_sms > kMaxSms) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv) & 15) ||
+        (reinterpret_cast<uintptr_t>(kv_scale) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+        (reinterpret_cast<uintptr_t>(out) & 7) || (reinterpret_cast<uintptr_t>(lse) & 3) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3) ||
+        (reinterpret_cast<uintptr_t>(sched_meta) & 3) || (reinterpret_cast<uintptr_t>(num_splits) & 3))
+        return MLA_ERR_MISALIGNED;
+    *wl = layout(B, s_q, *sh, num_sms);
+    if (workspace_bytes < wl->total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (static_cast<int64_t>(B) * s_q * H > INT32_MAX) return MLA_ERR_INVALID_ARG;
+    return MLA_OK;
+}
+
+// q viewed as [B * s_q * H rows][576 cols]; box 64 cols x (heads per CTA) rows.
+bool q_tensor_map(CUtensorMap *m, const uint16_t *q, int B, int s_q, int H, const Shape &sh)
+{
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(B) * s_q * H};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDQK) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sh.HG)};
+    return tensor_map(m, "q", CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
+mla_status_t decode_bf16(const uint16_t *q, const uint16_t *kv_cache, const int32_t *block_table,
+                         const int32_t *cache_seqlens, int B, int s_q, int H, int64_t num_blocks, int max_blocks,
+                         float softmax_scale, int num_sms, const int32_t *sched_meta, const int32_t *num_splits,
+                         void *workspace, size_t workspace_bytes, uint16_t *out, float *lse, void *stream,
+                         bool with_combine)
+{
+    clear_error();
+    Shape sh;
+    WorkspaceLayout wl;
+    const mla_status_t chk = check_decode_args(q, kv_cache, nullptr, false, block_table, cache_seqlens, B, s_q, H,
+                                               num_blocks, max_blocks, softmax_scale, num_sms, sched_meta,
+                                               num_splits, workspace, workspace_bytes, out, lse, &sh, &wl);
+    if (chk != MLA_OK) return chk;
+    // kv_cache viewed as [num_blocks][64 rows][576 cols]; box 64 cols x 64 rows x 1 block.
+    CUtensorMap kv_map, q_map;
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage),
+                                    static_cast<cuuint64_t>(num_blocks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK) * 2, static_cast<cuuint64_t>(kPage) * kDQK * 2};
+        const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kPage), 1};
+        if (!tensor_map(&kv_map, "kv", CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kv_cache, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+            return MLA_ERR_CUDA;
+    }
+    if (!q_tensor_map(&q_map, q, B, s_q, H, sh)) return MLA_ERR_CUDA;
+
+    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
+                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
+    const int grid = prm.num_tuples * sh.G;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // (the scale map is only read by the FP8 kernel; q_map stands in for it)
+    mla_status_t rc;
+    if (sh.N == 16) rc = launch_decode<16, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (sh.N == 32 && s_q == 1) rc = launch_decode<32, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (sh.N == 32) rc = launch_decode<32, 2, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 1) rc = launch_decode<64, 1, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 2) rc = launch_decode<64, 2, false>(kv_map, q_map, q_map, prm, grid, st);
+    else if (s_q == 4) rc = launch_decode<64, 4, false>(kv_map, q_map, q_map, prm, grid, st);
+    else rc = launch_decode<64, 8, false>(kv_map, q_map, q_map, prm, grid, st);
+    if (rc != MLA_OK || !with_combine) return rc;
+    return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
+                              stream);
+}
+
+mla_status_t decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
+                        const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q, int H,
+                        int64_t num_blocks, int max_blocks, float softmax_scale, int num_sms,
+                        const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
+                        size_t workspace_bytes, uint16_t *out, float *lse, void *stream, bool with_combine)
+{
+    clear_error();
+    Shape sh;
+    WorkspaceLayout wl;
+    const mla_status_t chk = check_decode_args(q, kv_codes, kv_scale, true, block_table, cache_seqlens, B, s_q, H,
+                                               num_blocks, max_blocks, softmax_scale, num_sms, sched_meta,
+                                               num_splits, workspace, workspace_bytes, out, lse, &sh, &wl);
+    if (chk != MLA_OK) return chk;
+    CUtensorMap kv_map, q_map, sc_map;
+    // codes viewed as [num_blocks][64 rows][576 bytes]; box 128 bytes x 64 rows x 1 block, 128-byte
+    // swizzled.  The rope group's box (columns 512..639) reads zeros past column 575.
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage),
+                                    static_cast<cuuint64_t>(num_blocks)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage) * kDQK};
+        const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(kPage), 1};
+        if (!tensor_map(&kv_map, "kv fp8", CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, kv_codes, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+            return MLA_ERR_CUDA;
+    }
+    // token scales viewed as [num_blocks][64]; box 64 x 1 block (256 bytes)
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kPage), static_cast<cuuint64_t>(num_blocks)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kPage) * 4};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kPage), 1};
+        if (!tensor_map(&sc_map, "kv scale", CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, kv_scale, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE))
+            return MLA_ERR_CUDA;
+    }
+    if (!q_tensor_map(&q_map, q, B, s_q, H, sh)) return MLA_ERR_CUDA;
+    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
+                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
+    const mla_status_t rc = launch_decode<16, 1, true>(kv_map, q_map, sc_map, prm, prm.num_tuples * sh.G,
+                                                       static_cast<cudaStream_t>(stream));
+    if (rc != MLA_OK || !with_combine) return rc;
+    return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
+                              stream);
+}
+
+}  // namespace host
+}  // namespace mla
 
 extern "C" {
 
@@ -1657,6 +1878,7 @@ size_t mla_decode_workspace_size(int B, int s_q, int H, int num_sms)
 mla_status_t mla_decode_metadata(const int32_t *cache_seqlens, int B, int s_q, int H, int num_sms,
                                  int32_t *sched_meta, int32_t *num_splits, void *stream)
 {
+    clear_error();
     if (!cache_seqlens || !sched_meta || !num_splits) return MLA_ERR_INVALID_ARG;
     if (B < 1 || B > kMaxBatch) return MLA_ERR_INVALID_ARG;
     Shape sh;
@@ -1677,6 +1899,7 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
                                 size_t workspace_bytes, int B, int s_q, int H, int num_sms, uint16_t *out,
                                 float *lse, void *stream)
 {
+    clear_error();
     if (!num_splits || !sched_meta || !workspace || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (B < 1 || B > kMaxBatch) return MLA_ERR_INVALID_ARG;
     Shape sh;
@@ -1708,80 +1931,13 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
 }
 
 mla_status_t mla_decode_attention(const uint16_t *q, const uint16_t *kv_cache, const int32_t *block_table,
-                        const int32_t *cache_seqlens, int B, int s_q, int H, int64_t num_blocks, int max_blocks,
-                        float softmax_scale, int num_sms, const int32_t *sched_meta, const int32_t *num_splits,
-                        void *workspace, size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
+                                  const int32_t *cache_seqlens, int B, int s_q, int H, int64_t num_blocks,
+                                  int max_blocks, float softmax_scale, int num_sms, const int32_t *sched_meta,
+                                  const int32_t *num_splits, void *workspace, size_t workspace_bytes, uint16_t *out,
+                                  float *lse, void *stream)
 {
-    if (!q || !kv_cache || !block_table || !cache_seqlens || !sched_meta || !num_splits || !workspace || !out ||
-        !lse)
-        return MLA_ERR_INVALID_ARG;
-    if (B < 1 || B > kMaxBatch || num_blocks < 1 || num_blocks > INT32_MAX || max_blocks < 1)
-        return MLA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
-    Shape sh;
-    if (!resolve(s_q, H, &sh)) return MLA_ERR_UNSUPPORTED_SHAPE;
-    if (num_sms < sh.G || num_sms > kMaxSms) return MLA_ERR_UNSUPPORTED_SHAPE;
-    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_cache) & 15) ||
-        (reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(out) & 7) ||
-        (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(block_table) & 3) ||
-        (reinterpret_cast<uintptr_t>(cache_seqlens) & 3) || (reinterpret_cast<uintptr_t>(sched_meta) & 3) ||
-        (reinterpret_cast<uintptr_t>(num_splits) & 3))
-        return MLA_ERR_MISALIGNED;
-    const WorkspaceLayout wl = layout(B, s_q, sh, num_sms);
-    if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
-    if (static_cast<int64_t>(B) * s_q * H > INT32_MAX) return MLA_ERR_INVALID_ARG;
-
-    EncodeTiledFn encode = encode_fn();
-    if (!encode) {
-        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
-        return MLA_ERR_CUDA;
-    }
-    // kv_cache viewed as [num_blocks][64 rows][576 cols]; box 64 cols x 64 rows x 1 block.
-    CUtensorMap kv_map, q_map;
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage),
-                                    static_cast<cuuint64_t>(num_blocks)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK) * 2, static_cast<cuuint64_t>(kPage) * kDQK * 2};
-        const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kPage), 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        const CUresult r = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(kv_cache), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(kv) failed: %d", static_cast<int>(r));
-            return MLA_ERR_CUDA;
-        }
-    }
-    // q viewed as [B * s_q * H rows][576 cols]; box 64 cols x (heads per CTA) rows.
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(B) * s_q * H};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDQK) * 2};
-        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sh.HG)};
-        const cuuint32_t estr[2] = {1, 1};
-        const CUresult r = encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(q), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(q) failed: %d", static_cast<int>(r));
-            return MLA_ERR_CUDA;
-        }
-    }
-
-    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
-                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
-    const int grid = prm.num_tuples * sh.G;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-    mla_status_t rc;
-    // (the scale map is only read by the FP8 kernel; q_map stands in for it)
-    if (sh.N == 16) rc = launch_decode<16, 1, false>(kv_map, q_map, q_map, prm, grid, st);
-    else if (sh.N == 32 && s_q == 1) rc = launch_decode<32, 1, false>(kv_map, q_map, q_map, prm, grid, st);
-    else if (sh.N == 32) rc = launch_decode<32, 2, false>(kv_map, q_map, q_map, prm, grid, st);
-    else if (s_q == 1) rc = launch_decode<64, 1, false>(kv_map, q_map, q_map, prm, grid, st);
-    else if (s_q == 2) rc = launch_decode<64, 2, false>(kv_map, q_map, q_map, prm, grid, st);
-    else if (s_q == 4) rc = launch_decode<64, 4, false>(kv_map, q_map, q_map, prm, grid, st);
-    else rc = launch_decode<64, 8, false>(kv_map, q_map, q_map, prm, grid, st);
-    return rc;
+    return decode_bf16(q, kv_cache, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks, softmax_scale,
+                       num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse, stream, false);
 }
 
 mla_status_t mla_decode(const uint16_t *q, const uint16_t *kv_cache, const int32_t *block_table,
@@ -1789,13 +1945,8 @@ mla_status_t mla_decode(const uint16_t *q, const uint16_t *kv_cache, const int32
                         float softmax_scale, int num_sms, const int32_t *sched_meta, const int32_t *num_splits,
                         void *workspace, size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
 {
-    const mla_status_t rc =
-        mla_decode_attention(q, kv_cache, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks,
-                             softmax_scale, num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse,
-                             stream);
-    if (rc != MLA_OK) return rc;
-    return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
-                              stream);
+    return decode_bf16(q, kv_cache, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks, softmax_scale,
+                       num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse, stream, true);
 }
 
 mla_status_t mla_decode_attention_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
@@ -1804,78 +1955,9 @@ mla_status_t mla_decode_attention_fp8(const uint16_t *q, const uint8_t *kv_codes
                                       const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
                                       size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
 {
-    if (!q || !kv_codes || !kv_scale || !block_table || !cache_seqlens || !sched_meta || !num_splits ||
-        !workspace || !out || !lse)
-        return MLA_ERR_INVALID_ARG;
-    if (B < 1 || B > kMaxBatch || num_blocks < 1 || num_blocks > INT32_MAX || max_blocks < 1)
-        return MLA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
-    Shape sh;
-    if (!resolve(s_q, H, &sh) || sh.N != 16 || s_q != 1) return MLA_ERR_UNSUPPORTED_SHAPE;
-    if (num_sms < sh.G || num_sms > kMaxSms) return MLA_ERR_UNSUPPORTED_SHAPE;
-    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv_codes) & 15) ||
-        (reinterpret_cast<uintptr_t>(kv_scale) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
-        (reinterpret_cast<uintptr_t>(out) & 7) || (reinterpret_cast<uintptr_t>(lse) & 3) ||
-        (reinterpret_cast<uintptr_t>(block_table) & 3) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3) ||
-        (reinterpret_cast<uintptr_t>(sched_meta) & 3) || (reinterpret_cast<uintptr_t>(num_splits) & 3))
-        return MLA_ERR_MISALIGNED;
-    const WorkspaceLayout wl = layout(B, s_q, sh, num_sms);
-    if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
-
-    EncodeTiledFn encode = encode_fn();
-    if (!encode) {
-        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
-        return MLA_ERR_CUDA;
-    }
-    CUtensorMap kv_map, q_map, sc_map;
-    // codes viewed as [num_blocks][64 rows][576 bytes]; box 128 bytes x 64 rows x 1 block, 128-byte
-    // swizzled.  The rope group's box (columns 512..639) reads zeros past column 575.
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage),
-                                    static_cast<cuuint64_t>(num_blocks)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(kPage) * kDQK};
-        const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(kPage), 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        const CUresult r = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(kv_codes), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(kv fp8) failed: %d", static_cast<int>(r));
-            return MLA_ERR_CUDA;
-        }
-    }
-    // token scales viewed as [num_blocks][64]; box 64 x 1 block (256 bytes)
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kPage), static_cast<cuuint64_t>(num_blocks)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kPage) * 4};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(kPage), 1};
-        const cuuint32_t estr[2] = {1, 1};
-        const CUresult r = encode(&sc_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(kv_scale), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(kv scale) failed: %d",
-                     static_cast<int>(r));
-            return MLA_ERR_CUDA;
-        }
-    }
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDQK), static_cast<cuuint64_t>(B) * s_q * H};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDQK) * 2};
-        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sh.HG)};
-        const cuuint32_t estr[2] = {1, 1};
-        const CUresult r = encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(q), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled(q) failed: %d", static_cast<int>(r));
-            return MLA_ERR_CUDA;
-        }
-    }
-    const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
-                                         softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
-    return launch_decode<16, 1, true>(kv_map, q_map, sc_map, prm, prm.num_tuples * sh.G,
-                                      static_cast<cudaStream_t>(stream));
+    return decode_fp8(q, kv_codes, kv_scale, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks,
+                      softmax_scale, num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse, stream,
+                      false);
 }
 
 mla_status_t mla_decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
@@ -1884,13 +1966,9 @@ mla_status_t mla_decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const fl
                             const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
                             size_t workspace_bytes, uint16_t *out, float *lse, void *stream)
 {
-    const mla_status_t rc =
-        mla_decode_attention_fp8(q, kv_codes, kv_scale, block_table, cache_seqlens, B, s_q, H, num_blocks,
-                                 max_blocks, softmax_scale, num_sms, sched_meta, num_splits, workspace,
-                                 workspace_bytes, out, lse, stream);
-    if (rc != MLA_OK) return rc;
-    return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
-                              stream);
+    return decode_fp8(q, kv_codes, kv_scale, block_table, cache_seqlens, B, s_q, H, num_blocks, max_blocks,
+                      softmax_scale, num_sms, sched_meta, num_splits, workspace, workspace_bytes, out, lse, stream,
+                      true);
 }
 
 mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_cache, const int32_t *block_table,
@@ -1899,6 +1977,7 @@ mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_c
                                          const int32_t *sched_meta, const int32_t *num_splits, uint16_t *out,
                                          float *lse, void *stream)
 {
+    clear_error();
     const size_t need = mla_decode_workspace_size(B, s_q, H, num_sms);
     if (need == 0) {
         if (B < 1 || B > kMaxBatch) return MLA_ERR_INVALID_ARG;
@@ -1917,8 +1996,11 @@ mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_c
                       num_sms, sched_meta, num_splits, ws, MLA_STATIC_WORKSPACE_BYTES, out, lse, stream);
 }
 
+void mla_debug_stall_cta(int cta) { g_debug_stall_cta.store(cta < 0 ? -1 : cta, std::memory_order_relaxed); }
+
 mla_status_t mla_get_device_error(const int32_t *sched_meta, int32_t *host_code, void *stream)
 {
+    clear_error();
     if (!sched_meta || !host_code) return MLA_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

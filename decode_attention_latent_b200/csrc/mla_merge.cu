@@ -23,6 +23,7 @@ namespace mla {
 namespace host {
 extern thread_local char g_last_error[256];
 mla_status_t cuda_fail(cudaError_t e, const char *what);
+void clear_error();
 }  // namespace host
 
 constexpr int kMergeMaxW = 64;
@@ -97,6 +98,7 @@ extern "C" mla_status_t mla_merge_states(const uint16_t *out_parts, const float 
                                          uint16_t *out, float *lse, void *stream)
 {
     using namespace mla;
+    host::clear_error();
     if (!out_parts || !lse_parts || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (W < 1 || W > kMergeMaxW || rows < 1 || rows > INT32_MAX) return MLA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(out_parts) | reinterpret_cast<uintptr_t>(out)) & 15) return MLA_ERR_MISALIGNED;

@@ -36,8 +36,13 @@
  *
  * Conventions for every call.
  *   - Pointers marked "device" are CUDA device pointers of the current
- *     device; the caller allocates and owns every buffer, the library
- *     allocates no device memory and keeps no state between calls.
+ *     device; the caller allocates and owns every buffer.  The library makes
+ *     no device allocation.  The one piece of device memory it holds is the
+ *     fixed MLA_STATIC_WORKSPACE_BYTES array behind
+ *     mla_decode_static_workspace, resident on every device that loads the
+ *     library and shared by every call of that entry point (see there).
+ *     Between calls it keeps only host-side state: encoded tensor maps,
+ *     cached by pointer and shape, and the test hook of mla_debug_stall_cta.
  *   - `stream` is a cudaStream_t (0 = the legacy default stream).  All
  *     launches are asynchronous on it; no call synchronises except
  *     mla_get_device_error.
@@ -179,10 +184,14 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
  *   - Returns MLA_ERR_WORKSPACE_TOO_SMALL, without launching, when the shape
  *     needs more than MLA_STATIC_WORKSPACE_BYTES
  *     (mla_decode_workspace_size(B, s_q, H, num_sms) tells); the message is in
- *     mla_last_error_message.
+ *     mla_last_error_message.  With 148 CTAs the three s_q = 1, 16-head
+ *     workloads of up to 16 sequences fit (4.9 to 5.4 MB); B = 32 at s_q = 2
+ *     (about 11.8 MB) and B = 64 at 128 heads (about 36 MB) are refused.
  *   - The first call on a device looks up the array's device address for that
  *     device (once; no allocation).  Make that first call before capturing any
- *     stream.
+ *     stream.  The address is kept for the life of the process: after a
+ *     cudaDeviceReset, or with another context made current on that device,
+ *     it is stale, so do not use this entry point across either.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Nothing in it needs to start at zero (every value read is written first
  *     by the same call), but calls whose kernels overlap on the GPU -- on two
@@ -221,6 +230,45 @@ mla_status_t mla_decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const fl
                             const int32_t *sched_meta, const int32_t *num_splits, void *workspace,
                             size_t workspace_bytes, uint16_t *out, float *lse, void *stream);
 
+/* Non-absorbed form.  The same latent cache, but each head attends with its
+ * own 192-wide keys and 128-wide values, decompressed from the latent rows
+ * tile by tile as "FlashMLA: compressing the KV cache to one eighth"
+ * (jsqmd.com), "FlashMLA compute flow", steps 1-5, describes (K_tile =
+ * C_KV_tile W_UK, V_tile = C_KV_tile W_UV, then S = Q K^T, online softmax,
+ * O += softmax(S) V).  For sequence b, query position i and head h, over
+ * the same visible tokens j as mla_decode (C_j = the 512 latent columns of
+ * token j's row, rope_j = its last 64 columns, cached already rotated and
+ * shared by every head):
+ *     k_j = [ W_UK[h] C_j (128) ,  rope_j (64) ],   v_j = W_UV[h] C_j (128)
+ *     out[b,i,h,:] = sum_j softmax(softmax_scale * <q[b,i,h,:], k_j>)_j v_j
+ *     lse[b,i,h]   = ln(sum_j exp(softmax_scale * <q[b,i,h,:], k_j>))
+ * The up-projections run on the tensor cores per 128-token tile (fp32
+ * accumulation); scores, softmax and the value sum stay in fp32.
+ *   q            device bf16 [B, s_q, H, 192]: 128 key columns, then 64 rope.
+ *   kv_cache, block_table, cache_seqlens, num_blocks, max_blocks,
+ *   softmax_scale: as for mla_decode (no schedule: each CTA takes one
+ *                sequence, one head and a fixed share of the tiles).
+ *   w_uk, w_uv   device bf16 [H, 128, 512], 16-byte aligned: row e of head h
+ *                holds the latent coefficients of key / value dimension e.
+ *   num_sms      SMs to size the split of each sequence for (148 on B200).
+ *   workspace    device, 256-byte aligned, workspace_bytes >=
+ *                mla_decode_naive_workspace_size(B, s_q, H, max_blocks,
+ *                num_sms); scratch for the splits' fp32 partial results.
+ *   error_word   device int32 [1], zeroed by the caller; the kernel ORs in
+ *                MLA_DEVERR_* bits (bad page-table entries, bad lengths,
+ *                timed-out waits) and never traps.
+ *   out          device bf16 [B, s_q, H, 128], 8-byte aligned (written).
+ *   lse          device fp32 [B, s_q, H] (written; natural log).
+ * Supported: s_q in {1, 2}; 1 <= H <= 128; 1 <= B <= 4096.  Launches the
+ * attention kernel and then its merge kernel on `stream`. */
+#define MLA_NAIVE_D 128   /* decompressed key / value width per head */
+size_t mla_decode_naive_workspace_size(int B, int s_q, int H, int max_blocks, int num_sms);
+mla_status_t mla_decode_naive(const uint16_t *q, const uint16_t *kv_cache, const uint16_t *w_uk,
+                              const uint16_t *w_uv, const int32_t *block_table, const int32_t *cache_seqlens,
+                              int B, int s_q, int H, int64_t num_blocks, int max_blocks, float softmax_scale,
+                              int num_sms, void *workspace, size_t workspace_bytes, int32_t *error_word,
+                              uint16_t *out, float *lse, void *stream);
+
 /* Merge of W partial attention states of the same output rows, each computed
  * over a disjoint range of the tokens -- in context-parallel decode, the
  * (out, lse) of W ranks that each hold a contiguous range of every sequence's
@@ -250,9 +298,19 @@ mla_status_t mla_get_device_error(const int32_t *sched_meta, int32_t *host_code,
 /* Static, human-readable name of a status code. */
 const char *mla_status_string(mla_status_t status);
 
-/* Text of the last MLA_ERR_CUDA raised on the calling thread (the failing
- * CUDA call and its error string); "" if none.  Owned by the library. */
+/* Text explaining the last error status of a call on the calling thread: the
+ * failing CUDA call and its error string for MLA_ERR_CUDA, and the sizes for
+ * the MLA_ERR_WORKSPACE_TOO_SMALL of mla_decode_static_workspace.  Every
+ * entry point clears it when called, so it never outlives the next call; ""
+ * if the last call set none.  Owned by the library. */
 const char *mla_last_error_message(void);
+
+/* Test hook for the failure path of the bounded device waits: from the next
+ * decode launch on, CTA `cta` announces its first cache load without issuing
+ * it, so its waits run out after their time limit (about 2 s), set
+ * MLA_DEVERR_TIMEOUT and end; -1 turns the hook off (the default).
+ * Process-wide; not for use in production. */
+void mla_debug_stall_cta(int cta);
 
 #ifdef __cplusplus
 }

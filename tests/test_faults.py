@@ -1,13 +1,16 @@
 """Failure detection on the GPU without a fault.
 
-A CTA whose first cache chunk is announced but never loaded (the library's
-MLA_DEBUG_STALL_CTA test hook) must end its bounded waits after their time
+A CTA whose first cache load is announced but never issued (the library's
+mla_debug_stall_cta test hook) must end its bounded waits after their time
 limit, report MLA_DEVERR_TIMEOUT in the device error word, release its TMEM
 and exit; the context must stay usable, so the next call on the same process
-returns a clean error word and results equal to the oracle's.  The check runs
-in a child process so the hook's environment variable never reaches other
-tests.  Invalid data (a bad page-table entry, a schedule built for another
-shape) is covered in test_parity.py.
+(after mla_decode_metadata has reset sched_meta, as the header asks after a
+device error) returns a clean error word and results equal to the oracle's.
+Both the bf16 kernel and the FP8-cache kernel (whose first staging unit is the
+one withheld) are checked.  Each check runs in a child process so the hook
+never reaches other tests.  Invalid data (a bad page-table entry, a schedule
+built for another shape, a stale completion counter) is covered in
+test_parity.py.
 """
 import os
 import subprocess
@@ -32,22 +35,34 @@ import oracle
 dev = torch.device("cuda", 0)
 inp = mi.small(B=3, s_q=1, H=16, seqlens=[900, 300, 2000], seed=900)
 q, kv, bt, sl = (x.to(dev) for x in (inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens))
+if FP8:
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=901)
+    codes, scales = cache.codes.to(dev), cache.scale.to(dev)
 
 
 def run():
     sched, splits = mla.decode_metadata(sl, 1, 16, 8)
-    out, lse = mla.decode(q, kv, bt, sl, inp.scale, sched_meta=sched, num_splits=splits, num_sms_=8)
+    if FP8:
+        out, lse = mla.decode_fp8(q, codes, scales, bt, sl, inp.scale, sched_meta=sched, num_splits=splits,
+                                  num_sms_=8)
+    else:
+        out, lse = mla.decode(q, kv, bt, sl, inp.scale, sched_meta=sched, num_splits=splits, num_sms_=8)
     return out, lse, mla.get_device_error(sched)
 
 
-os.environ["MLA_DEBUG_STALL_CTA"] = "3"   # CTA 3 of 8 owns tiles 12..15 of the 27
+mla.debug_stall_cta(3)   # CTA 3 of 8 owns tiles 12..15 of the 27
 _, _, err = run()
 print("stalled call error word", err)
 assert err & mla.DEVERR_TIMEOUT, err
-del os.environ["MLA_DEBUG_STALL_CTA"]
+mla.debug_stall_cta(-1)
 out, lse, err = run()
 assert err == 0, err
-ref_out, ref_lse = oracle.default().direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+orc = oracle.default()
+if FP8:
+    ref_out, ref_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens,
+                                      inp.scale)
+else:
+    ref_out, ref_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
 g_out = out.float().cpu().numpy()
 g_lse = lse.cpu().numpy()
 ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref_out), 1e-30))) - 7)  # one bf16 ulp
@@ -57,10 +72,10 @@ print("ok")
 '''
 
 
-def test_stalled_cta_times_out_and_context_survives():
+@pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "fp8"])
+def test_stalled_cta_times_out_and_context_survives(fp8):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    env = {k: v for k, v in os.environ.items() if k != "MLA_DEBUG_STALL_CTA"}
-    r = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\n" + CHILD], capture_output=True, text=True,
-                       timeout=300, env=env)
+    r = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\nFP8 = {fp8!r}\n" + CHILD], capture_output=True,
+                       text=True, timeout=300)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

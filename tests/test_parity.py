@@ -2,12 +2,16 @@
 
 Tolerances (from the arithmetic: bf16 inputs, fp32 accumulation, bf16 P and
 output):
-  out  |gpu - ref| <= 1.5e-2 + ulp_bf16(ref)   (1.5e-2 absolute plus one bf16
-       ulp of the reference, 2^(floor(log2|ref|) - 7): the weights P are
+  out  |gpu - ref| <= 1.5e-2 wherever |ref| < 1 (the stated bound, plain), and
+       <= 1.5e-2 + ulp_bf16(ref) where |ref| >= 1: one bf16 ulp of the
+       reference, 2^(floor(log2|ref|) - 7), added because the weights P are
        rounded to bf16 before the output MMA, which alone can move a near
        one-hot output by up to 2^-9 |V|, and the output itself is rounded to
-       bf16; for |ref| < 0.6 this is within 4e-3 of the plain 1.5e-2 bound)
-       and relative RMSE  sqrt(sum (gpu-ref)^2 / sum ref^2) <= 5e-3;
+       bf16 (half an ulp, already 0.0156 at |out| = 4).  Outputs of N(0, 1)
+       inputs over more than a few tokens stay below 1, so the 16- and
+       128-head workloads are held to the plain bound everywhere; the x20
+       outlier workload and contexts of a few tokens reach |out| >= 1.
+       Relative RMSE  sqrt(sum (gpu-ref)^2 / sum ref^2) <= 5e-3;
   lse  |gpu - ref| <= 1e-3, and -inf exactly where the reference is -inf.
 Integer work (the schedule) is compared exactly.
 """
@@ -32,6 +36,23 @@ def ulp_bf16(x):
     """Spacing of bf16 numbers at |x| (8 significant bits)."""
     a = np.abs(np.asarray(x, dtype=np.float64))
     return np.exp2(np.floor(np.log2(np.maximum(a, 1e-30))) - 7)
+
+
+def out_bound(ref):
+    """Elementwise bound on |gpu - ref|: the plain 1.5e-2 below |ref| = 1,
+    plus one bf16 ulp of the reference from there on."""
+    ref = np.asarray(ref, dtype=np.float64)
+    return np.where(np.abs(ref) < 1.0, ATOL, ATOL + ulp_bf16(ref))
+
+
+def error_stats(g_out, g_lse, r_out, r_lse):
+    """max |out err|, relative RMSE of out, max |lse err| (finite rows)."""
+    err = np.abs(g_out.astype(np.float64) - r_out)
+    den = float(np.sum(r_out.astype(np.float64) ** 2))
+    rmse = math.sqrt(float(np.sum(err ** 2)) / den) if den > 0 else 0.0
+    fin = np.isfinite(r_lse)
+    lerr = float(np.abs(g_lse[fin] - r_lse[fin]).max()) if fin.any() else 0.0
+    return float(err.max()), rmse, lerr
 
 
 @pytest.fixture(scope="module")
@@ -67,7 +88,7 @@ def compare(g_out, g_lse, r_out, r_lse, seqs=None, what=""):
     assert np.all(g_lse[~fin] == -np.inf), f"{what}: empty rows must have lse = -inf"
     assert np.all(g_out[~fin] == 0), f"{what}: empty rows must have out = 0"
     err = np.abs(g_out - r_out)
-    bound = ATOL + ulp_bf16(r_out)
+    bound = out_bound(r_out)
     worst = np.unravel_index(np.argmax(err - bound), err.shape)
     assert np.all(err <= bound), (f"{what}: out err {err[worst]:.4e} > {bound[worst]:.4e} at {worst} "
                                   f"(gpu {g_out[worst]:.6f} ref {r_out[worst]:.6f})")
@@ -241,6 +262,29 @@ def test_malformed_schedule_range_is_detected(dev):
     mla.decode(inp.q.to(dev), inp.kv_cache.to(dev), inp.block_table.to(dev), sl, inp.scale,
                sched_meta=sched, num_splits=splits, num_sms_=16)
     assert mla.get_device_error(sched) & mla.DEVERR_SCHEDULE
+
+
+@pytest.mark.parametrize("s_q,H,n_sms", [(1, 16, 148), (2, 16, 17), (1, 128, 148), (4, 32, 7)])
+def test_separate_attention_and_combine_calls(dev, orc, s_q, H, n_sms):
+    """mla_decode_attention and mla_decode_combine called apart (the
+    pieces of split sequences left in a caller-held workspace, then merged)
+    against the oracle, and bitwise against mla_decode."""
+    lens = [0, 5, 700, 129, 4000, 64]
+    inp = mi.small(B=len(lens), s_q=s_q, H=H, seqlens=lens, seed=850 + H + s_q, tail_fill=float("nan"))
+    q, kv, bt, sl = (x.to(dev) for x in (inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens))
+    sched, splits = mla.decode_metadata(sl, s_q, H, n_sms)
+    ws = torch.empty(mla.workspace_size(inp.B, s_q, H, n_sms), dtype=torch.uint8, device=dev)
+    out = torch.full((inp.B, s_q, H, 512), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((inp.B, s_q, H), float("nan"), dtype=torch.float32, device=dev)
+    mla.decode(q, kv, bt, sl, inp.scale, sched_meta=sched, num_splits=splits, num_sms_=n_sms, workspace=ws,
+               out=out, lse=lse, combine=False)
+    mla.decode_combine(splits, sched, ws, inp.B, s_q, H, out, lse, num_sms_=n_sms)
+    assert mla.get_device_error(sched) == 0
+    g_out, g_lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"two-kernel s_q={s_q} H={H}")
+    one = run_gpu(inp, dev, n_sms=n_sms)
+    assert np.array_equal(one[0], g_out) and np.array_equal(one[1], g_lse), "separate calls differ from mla_decode"
 
 
 # ---------------------------------------------------- schedule (integers)
