@@ -766,6 +766,78 @@ def run_fp8(args):
     return 0
 
 
+def run_naive(args):
+    """The non-absorbed form (mla_decode_naive) on the workload's cache, one
+    GPU: per-head up-projections of every tile on the tensor cores, so the
+    roofline is the bf16 tensor peak over its algorithmic FLOPs; the error
+    against the oracle's non-absorbed form on a bounded sample (the fp64
+    decompression of every token is too slow for the whole workload)."""
+    import numpy as np
+
+    import decode_attention_latent_b200 as mla
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mla.load_library()
+    w = selected_workload(args)
+    if w.s_q > 2:
+        raise SystemExit("the non-absorbed form takes s_q <= 2")
+    inp = mi.make_inputs(w, seed=0)
+    nv = mi.naive_inputs(w.B, w.s_q, w.H, seed=1)
+    q, kv, wk, wv = nv.q.to(dev), inp.kv_cache.to(dev), nv.w_uk.to(dev), nv.w_uv.to(dev)
+    bt, sl = inp.block_table.to(dev), inp.cache_seqlens.to(dev)
+    out, lse, err = mla.decode_naive(q, kv, wk, wv, bt, sl, inp.scale)
+    for _ in range(max(3, args.warmup)):
+        mla.decode_naive(q, kv, wk, wv, bt, sl, inp.scale, out=out, lse=lse, error_word=err)
+    torch.cuda.synchronize(dev)
+    assert int(err.item()) == 0
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(0).start()
+    time.sleep(0.3)
+    t0 = time.time()
+    for k in range(K):
+        ev[k][0].record(); mla.decode_naive(q, kv, wk, wv, bt, sl, inp.scale, out=out, lse=lse, error_word=err)
+        ev[k][1].record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop(t0, time.time())
+    assert int(err.item()) == 0
+    call_us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    flops = mi.naive_algorithmic_flops(inp)
+    _, _, tc, tc_src = measured_peaks()
+    achieved = flops / (call_us * 1e-6) / 1e12
+    acc = None
+    if not args.no_cpu_baseline:
+        import oracle
+        # bounded sample: the first two sequences cut to 1024 tokens, same q and matrices
+        sub = mi.Inputs(q=inp.q[:2], kv_cache=inp.kv_cache, block_table=inp.block_table[:2],
+                        cache_seqlens=inp.cache_seqlens[:2].clamp(max=1024), scale=inp.scale)
+        g_out, g_lse, _ = mla.decode_naive(q[:2].contiguous(), kv, wk, wv, bt[:2].contiguous(),
+                                           sub.cache_seqlens.to(dev), inp.scale)
+        torch.cuda.synchronize(dev)
+        r_out, r_lse = oracle.default().naive(nv.q[:2], inp.kv_cache, nv.w_uk, nv.w_uv, sub.block_table,
+                                              sub.cache_seqlens, inp.scale)
+        acc = accuracy(g_out.float().cpu().numpy(), g_lse.cpu().numpy(), r_out, r_lse, None, 2)
+        acc["sequences"] = "2 sequences cut to their first 1024 tokens"
+    line = {
+        "metric": "MLA decode, non-absorbed form (per-tile up-projection) us/call", "value": call_us,
+        "unit": "us/call", "n_gpus": 1, "steps": K, "warmup": args.warmup, "higher_is_better": False,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "s_q": w.s_q, "H": w.H, "kv_bytes": int(inp.kv_cache.numel() * 2),
+                   "weights": "w_uk, w_uv [H, 128, 512] bf16, N(0, 1/512)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc, "unit": "TFLOP/s", "frac": achieved / tc,
+                     "peak_source": tc_src, "frac_of_sustained": achieved / sustained_tflops(),
+                     "algorithmic_flops_per_launch": flops, "traffic": None,
+                     "kernel": f"mla_naive_kernel<{w.s_q}>"},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if acc is not None:
+        line["accuracy"] = acc
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -777,6 +849,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="cut the workload to its first BATCH sequences (profiler captures on a smaller case)")
     ap.add_argument("--fp8", action="store_true", help="the same workload over an FP8 (e4m3) cache (H = 16, s_q = 1)")
+    ap.add_argument("--naive", action="store_true",
+                    help="the non-absorbed form (per-tile up-projection) on the same workload")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="W",
                     help="time one rank of a W-way context-parallel decode on one GPU (s_q = 1 workloads)")
     args = ap.parse_args(argv)
@@ -785,6 +859,8 @@ def main(argv=None):
         return run_context_parallel_rank(args)
     if args.fp8 and args.impl == "ours":
         return run_fp8(args)
+    if args.naive and args.impl == "ours":
+        return run_naive(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_ours(args, world, rank, local)

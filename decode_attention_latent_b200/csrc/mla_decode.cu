@@ -230,18 +230,114 @@ __device__ int last_at_or_below(const int *prefix, int B, int x)
     return lo;
 }
 
+// Header and error word of the schedule (thread 0).
+__device__ __forceinline__ void write_sched_header(int32_t *sched, int bad, int B, int s_q, int H, int num_sms,
+                                                   int num_tuples, int G, int per, int total, int total_splits)
+{
+    sched[0] = bad ? MLA_DEVERR_SEQLEN : 0;
+    sched[1] = kSchedMagic;
+    sched[2] = B;
+    sched[3] = s_q;
+    sched[4] = H;
+    sched[5] = num_sms;
+    sched[6] = num_tuples;
+    sched[7] = G;
+    sched[8] = per;
+    sched[9] = total;
+    sched[10] = total_splits;
+    for (int k = 11; k < kSchedHeader; ++k) sched[k] = 0;
+}
+
+// Work range of CTA group k: {b0, first tile in b0, b1, end tile in b1,
+// piece index within b0}, or {-1, 0, -1, 0, 0} past the last tile.
+__device__ __forceinline__ void write_sched_entry(int32_t *sched, int k, int per, int total, int b0, int pre_b0,
+                                                  int b1, int pre_b1)
+{
+    int32_t *e = sched + kSchedHeader + k * kSchedEntry;
+    const int start = k * per;
+    if (start >= total) {
+        e[0] = -1; e[1] = 0; e[2] = -1; e[3] = 0; e[4] = 0; e[5] = 0; e[6] = 0; e[7] = 0;
+        return;
+    }
+    const int end = min(start + per, total);
+    e[0] = b0;
+    e[1] = start - pre_b0;
+    e[2] = b1;
+    e[3] = end - pre_b1;
+    e[4] = k - pre_b0 / per;  // index of this group's piece of sequence b0
+    e[5] = 0; e[6] = 0; e[7] = 0;
+}
+
+// Batches of at most 32 sequences: one warp, prefix sums by shuffles, no
+// block barrier.  Lane b holds sequence b.
+__device__ void metadata_warp(const int32_t *__restrict__ seqlens, int B, int s_q, int H, int num_sms,
+                              int num_tuples, int G, int32_t *__restrict__ sched, int32_t *__restrict__ split_base,
+                              int *pre_s)
+{
+    const int lane = threadIdx.x;
+    int L = lane < B ? seqlens[lane] : 0;
+    const bool bad = __any_sync(0xffffffffu, L < 0);
+    L = max(L, 0);
+    const int nt = tiles_of(L);
+    int inc = nt;  // inclusive prefix of tiles
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    const int pre = inc - nt;  // exclusive prefix: first tile of sequence `lane`
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    const int per = total > 0 ? (total + num_tuples - 1) / num_tuples : 1;
+    pre_s[lane] = pre;
+    __syncwarp();
+    for (int k = lane; k < num_tuples; k += 32) {
+        const int start = k * per;
+        if (start >= total) {
+            write_sched_entry(sched, k, per, total, 0, 0, 0, 0);
+            continue;
+        }
+        const int end = min(start + per, total);
+        const int b0 = last_at_or_below(pre_s, B, start);
+        const int b1 = last_at_or_below(pre_s, B, end - 1);
+        write_sched_entry(sched, k, per, total, b0, pre_s[b0], b1, pre_s[b1]);
+    }
+    const int ns = nt > 0 ? (pre + nt - 1) / per - pre / per + 1 : 0;
+    int ninc = ns;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ninc, o);
+        if (lane >= o) ninc += y;
+    }
+    if (lane < B) split_base[lane] = ninc - ns;
+    const int total_splits = __shfl_sync(0xffffffffu, ninc, 31);
+    if (lane == 0) {
+        split_base[B] = total_splits;
+        write_sched_header(sched, bad, B, s_q, H, num_sms, num_tuples, G, per, total, total_splits);
+    }
+}
+
+// The schedule in shared memory sized to the batch (2 (B + 1) + 33 ints,
+// dynamic), so that for small batches the block fits on an SM beside an
+// attention CTA and every attention CTA can start at once.
 __global__ void __launch_bounds__(kMetaThreads, 1)
 mla_metadata_kernel(const int32_t *__restrict__ seqlens, int B, int s_q, int H, int num_sms,
                     int num_tuples, int G, int32_t *__restrict__ sched, int32_t *__restrict__ split_base)
 {
-    __shared__ int prefix[kMaxBatch + 1];
-    __shared__ int nsplit[kMaxBatch + 1];
-    __shared__ int warp_sums[32];
-    __shared__ int bad_len;
-    const int tid = threadIdx.x;
     // The attention grid may become resident now: it runs its prologue and
     // then waits for this grid to complete before reading the schedule.
     ptx::griddep_launch_dependents();
+    extern __shared__ uint8_t smem_raw[];
+    if (B <= 32) {
+        if (threadIdx.x < 32)
+            metadata_warp(seqlens, B, s_q, H, num_sms, num_tuples, G, sched, split_base,
+                          reinterpret_cast<int *>(smem_raw));
+        return;
+    }
+    int *prefix = reinterpret_cast<int *>(smem_raw);  // [B + 1]
+    int *nsplit = prefix + (B + 1);   // [B + 1]
+    int *warp_sums = nsplit + (B + 1);  // [32]
+    int &bad_len = warp_sums[32];
+    const int tid = threadIdx.x;
     if (tid == 0) bad_len = 0;
     __syncthreads();
     for (int b = tid; b < B; b += kMetaThreads) {
@@ -259,21 +355,15 @@ mla_metadata_kernel(const int32_t *__restrict__ seqlens, int B, int s_q, int H, 
     const int per = total > 0 ? (total + num_tuples - 1) / num_tuples : 1;
 
     for (int k = tid; k < num_tuples; k += kMetaThreads) {
-        int32_t *e = sched + kSchedHeader + k * kSchedEntry;
         const int start = k * per;
         if (start >= total) {
-            e[0] = -1; e[1] = 0; e[2] = -1; e[3] = 0; e[4] = 0; e[5] = 0; e[6] = 0; e[7] = 0;
+            write_sched_entry(sched, k, per, total, 0, 0, 0, 0);
             continue;
         }
         const int end = min(start + per, total);
         const int b0 = last_at_or_below(prefix, B, start);
         const int b1 = last_at_or_below(prefix, B, end - 1);
-        e[0] = b0;
-        e[1] = start - prefix[b0];
-        e[2] = b1;
-        e[3] = end - prefix[b1];
-        e[4] = k - prefix[b0] / per;  // index of this group's piece of sequence b0
-        e[5] = 0; e[6] = 0; e[7] = 0;
+        write_sched_entry(sched, k, per, total, b0, prefix[b0], b1, prefix[b1]);
     }
     for (int b = tid; b < B; b += kMetaThreads) {
         const int nt = prefix[b + 1] - prefix[b];
@@ -284,18 +374,7 @@ mla_metadata_kernel(const int32_t *__restrict__ seqlens, int B, int s_q, int H, 
     for (int b = tid; b < B; b += kMetaThreads) split_base[b] = nsplit[b];
     if (tid == 0) {
         split_base[B] = total_splits;
-        sched[0] = bad_len ? MLA_DEVERR_SEQLEN : 0;
-        sched[1] = kSchedMagic;
-        sched[2] = B;
-        sched[3] = s_q;
-        sched[4] = H;
-        sched[5] = num_sms;
-        sched[6] = num_tuples;
-        sched[7] = G;
-        sched[8] = per;
-        sched[9] = total;
-        sched[10] = total_splits;
-        for (int k = 11; k < kSchedHeader; ++k) sched[k] = 0;
+        write_sched_header(sched, bad_len, B, s_q, H, num_sms, num_tuples, G, per, total, total_splits);
     }
 }
 
@@ -728,8 +807,6 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;
     uint32_t cc = 0, v = 0;
-    uint32_t c8 = 0;         // FP8 staging unit uses so far
-    bool vt_ok = true;       // FP8: a failed V^T wait, carried to the next agreement
     bool ok = true;
     // ldmatrix row addresses: lane -> (matrix mi, row rr).  Matrices 0 and 2
     // take tokens {0,1,4,5,8,9,12,13} of a 16-token group, matrices 1 and 3
@@ -815,100 +892,6 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
                     }
             };
             uint32_t ra[64], rb[64];
-            if constexpr (F8) {
-                // Unit k of the tile becomes ring slot cc + k (chunks 2k, 2k + 1;
-                // the rope group fills the first chunk of slot cc + 4): thread
-                // row r converts its token's 128 e4m3 codes to bf16 (exactly),
-                // in the swizzled layout the TMA gives bf16 chunks; then the
-                // slot is handed to the score MMA (full barrier, four warp
-                // arrivals) and the unit back to the producer.  The token's
-                // scale goes to the softmax, which applies it in fp32 to the
-                // token's scores and to its weights in P^T.
-                auto convert = [&](int k) -> bool {
-                    const uint32_t u8 = c8 + k;
-                    const int us = static_cast<int>(u8 % kF8Ring);
-                    if (!warp_wait(sm.bar(kBarF8Full + us), (u8 / kF8Ring) & 1, sm.abort_flag, p.err)) return false;
-                    const uint32_t su = cc + k;
-                    const int slot = static_cast<int>(su % R);
-                    if (!warp_wait(sm.bar(kBarEmpty + slot), ((su / R) & 1) ^ 1, sm.abort_flag, p.err)) return false;
-                    const uint32_t src = sm.f8 + us * kF8Unit;
-                    const uint32_t r = static_cast<uint32_t>(32 * q + lane);
-                    const uint32_t sw = r & 7u;
-                    if (k == 0) {
-                        // this row's token scale, for the softmax of this tile
-                        const uint32_t tile = c8 / kF8Units, sbuf = tile % kScBufs;
-                        if (!warp_wait(sm.bar(kBarScEmpty + sbuf), ((tile / kScBufs) & 1) ^ 1, sm.abort_flag, p.err))
-                            return false;
-                        sm.tscale[sbuf * 128 + r] = ptx::ld_shared_f32(src + kF8ScaleOff + 4u * r);
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(sm.bar(kBarScFull + sbuf));
-                    }
-                    const uint32_t dst = sm.slot(slot) + r * 128u;
-                    const int nlu = (k == kF8Units - 1) ? 4 : 8;  // the rope group is 64 columns
-#pragma unroll
-                    for (int lu = 0; lu < 8; ++lu) {
-                        if (lu < nlu) {
-                            const uint4 wv = ptx::ld_shared_v4(src + r * 128u + ((static_cast<uint32_t>(lu) ^ sw) << 4));
-                            const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-                            uint32_t o[8];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float2 lo = ptx::e4m3x2_to_float2(words[i], false);
-                                const float2 hi = ptx::e4m3x2_to_float2(words[i], true);
-                                o[2 * i] = ptx::pack_bf16x2(lo.x, lo.y);  // exact: e4m3 values are bf16 values
-                                o[2 * i + 1] = ptx::pack_bf16x2(hi.x, hi.y);
-                            }
-                            const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
-                            const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
-                            ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
-                            ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
-                        }
-                    }
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::mbar_arrive(sm.bar(kBarFull + slot));
-                        ptx::mbar_arrive(sm.bar(kBarF8Empty + us));
-                    }
-                    return true;
-                };
-                const uint32_t s0 = cc % R;
-                // The four converter warps agree (named barrier 2) after every
-                // conversion, so every row of a slot is written before any warp
-                // reads it transposed, and a failed wait ends all four together.
-                bool okc = convert(0);
-                if (!(ok = ptx::named_bar_and(2, 128, okc && vt_ok))) break;
-                load_chunk(0, s0, ra);
-                release(s0, ra);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t(&cur)[64] = (j & 1) ? rb : ra;
-                    uint32_t(&nxt)[64] = (j & 1) ? ra : rb;
-                    if (j < 3) {
-                        okc = convert(j + 1);
-                        if (j == 2) okc = convert(kF8Units - 1) && okc;
-                        if (!(ok = ptx::named_bar_and(2, 128, okc && vt_ok))) break;
-                        const uint32_t sn = (cc + static_cast<uint32_t>(j) + 1u) % R;
-                        load_chunk(j + 1, sn, nxt);
-                        release(sn, nxt);
-                    }
-                    const uint32_t vb = v % NVT, vu = v / NVT;
-                    if (vu >= 1) vt_ok = warp_wait(sm.bar(kBarVtEmpty + vb), (vu & 1) ^ 1, sm.abort_flag, p.err) && vt_ok;
-                    if (vt_ok) {
-                        ptx::tc_fence_after();
-                        store_chunk(vb, cur);
-                        ptx::tmem_wait_st();
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(sm.bar(kBarVtFull + vb));
-                    }
-                    ++v;
-                }
-                if (!ok) break;
-                cc += C::SPT;
-                c8 += kF8Units;
-                continue;
-            }
             uint32_t slot_a = 0, slot_b = 0;
             if (!(ok = wait_chunk(0, slot_a))) break;
             load_chunk(0, slot_a, ra);
@@ -974,6 +957,72 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     uint32_t it = 0;   // tiles processed
     bool ok = true;
 
+    // FP8 cache: these four warps, idle for most of a tile at 16 query
+    // columns, widen the tile's five e4m3 staging units into its five bf16
+    // ring slots (thread = token row r: 128 codes -> bf16, exactly, in the
+    // swizzled layout TMA gives bf16 chunks), one tile ahead of their own
+    // softmax, so the transposer warps only transpose.  The tile's token
+    // scales go to a small ring read by the softmax (Smem::tscale).
+    uint32_t c8 = 0, cc8 = 0;            // staging units / ring slot uses converted
+    uint32_t nconv = 0, total_tiles = 0;  // tiles converted / tiles of this CTA
+    bool conv_ok = true;
+    if constexpr (F8) {
+        for (int b = w.b0; b <= w.b1; ++b) {
+            const int nt = tiles_of(max(0, __ldg(p.seqlens + b)));
+            const int tb = (b == w.b0) ? w.t0 : 0;
+            const int te = min((b == w.b1) ? w.t1 : nt, nt);
+            total_tiles += static_cast<uint32_t>(max(0, te - tb));
+        }
+    }
+    auto convert_tile = [&]() {
+        const uint32_t R = static_cast<uint32_t>(p.ring);
+        const uint32_t r = static_cast<uint32_t>(32 * wq + lane);
+        const uint32_t sw = r & 7u;
+#pragma unroll 1
+        for (int k = 0; k < kF8Units; ++k) {
+            const uint32_t u8 = c8 + k;
+            const int us = static_cast<int>(u8 % kF8Ring);
+            conv_ok = conv_ok && warp_wait(sm.bar(kBarF8Full + us), (u8 / kF8Ring) & 1, sm.abort_flag, p.err);
+            const uint32_t su = cc8 + k;
+            const int slot = static_cast<int>(su % R);
+            conv_ok = conv_ok && warp_wait(sm.bar(kBarEmpty + slot), ((su / R) & 1) ^ 1, sm.abort_flag, p.err);
+            if (!conv_ok) continue;
+            const uint32_t src = sm.f8 + us * kF8Unit;
+            if (k == 0) sm.tscale[(nconv % kScBufs) * 128 + r] = ptx::ld_shared_f32(src + kF8ScaleOff + 4u * r);
+            const uint32_t dst = sm.slot(slot) + r * 128u;
+            const int nlu = (k == kF8Units - 1) ? 4 : 8;  // the rope group is 64 columns
+#pragma unroll
+            for (int lu = 0; lu < 8; ++lu) {
+                if (lu < nlu) {
+                    const uint4 wv = ptx::ld_shared_v4(src + r * 128u + ((static_cast<uint32_t>(lu) ^ sw) << 4));
+                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 lo = ptx::e4m3x2_to_float2(words[i], false);
+                        const float2 hi = ptx::e4m3x2_to_float2(words[i], true);
+                        o[2 * i] = ptx::pack_bf16x2(lo.x, lo.y);  // exact: e4m3 values are bf16 values
+                        o[2 * i + 1] = ptx::pack_bf16x2(hi.x, hi.y);
+                    }
+                    const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
+                    const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
+                    ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
+                    ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(sm.bar(kBarFull + slot));
+                ptx::mbar_arrive(sm.bar(kBarF8Empty + us));
+            }
+        }
+        c8 += kF8Units;
+        cc8 += C::SPT;
+        ++nconv;
+        ptx::named_bar_sync(1, 128);  // the tile's token scales, from every warp, before any reads them
+    };
+
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
         const int L = max(0, __ldg(p.seqlens + b));
         const int nt = tiles_of(L);
@@ -988,6 +1037,11 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         bool wait_ok = true;  // a failed wait is carried to the next agreement point
 
         for (int t = tb; t < te; ++t) {
+            if constexpr (F8) {
+                // keep the converted tiles one ahead of this softmax (tile it + 1)
+                while (nconv < total_tiles && nconv <= it + 1) convert_tile();
+                wait_ok = wait_ok && conv_ok;
+            }
             const uint32_t sb = it % C::NS, su = it / C::NS;
             wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
             ptx::tc_fence_after();
@@ -1009,8 +1063,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             // past the visible tokens, so their zero weights stay zero)
             float tsc[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
             if constexpr (F8) {
-                const uint32_t sbuf = it % kScBufs;
-                wait_ok = wait_bounded(sm.bar(kBarScFull + sbuf), (it / kScBufs) & 1, sm.abort_flag, p.err) && wait_ok;
+                const uint32_t sbuf = it % kScBufs;  // written by convert_tile, behind a named barrier
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -1018,8 +1071,6 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                         const int row = 32 * wq + r8 + 16 * hf + 8 * jj;
                         tsc[hf][jj] = (tok0 + 16 * hf + 8 * jj < nvis0) ? sm.tscale[sbuf * 128 + row] : 0.f;
                     }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(sm.bar(kBarScEmpty + sbuf));
             }
             float d[2][NG][4];
             bool flag = first || !wait_ok;
@@ -1308,18 +1359,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
 
 // =============================================================== combine
 // One 128-thread block per output row (b, i, h) of a sequence cut into pieces.
-// Each thread owns four latent dims and issues the loads of a batch of pieces
-// together, so the partials are fetched with all loads in flight instead of
-// one piece at a time; 64 registers a thread keep 8 blocks resident per SM.  Launched as a programmatic dependent of the attention kernel: it may
-// become resident early and waits in hardware for that grid to finish.
+// Each thread owns four latent dims and issues the loads of a batch of 20
+// pieces together (the ~19 pieces of a 64K-context sequence split over 148
+// SMs in one memory round trip instead of three of 8).  Launched as a
+// programmatic dependent of the attention kernel: it may become resident
+// early and waits in hardware for that grid to finish.
 constexpr int kCombineThreads = 128;
 
-__global__ void __launch_bounds__(kCombineThreads, 8)
+__global__ void __launch_bounds__(kCombineThreads, 4)
 mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restrict__ ws_o,
                    const float *__restrict__ ws_lse, int B, int s_q, int H, int HG, int G, int max_pieces,
                    uint16_t *__restrict__ out, float *__restrict__ lse, int32_t *__restrict__ err)
 {
-    constexpr int kBatch = 8;  // pieces whose loads are in flight together
+    constexpr int kBatch = 20;  // pieces whose loads are in flight together
     ptx::griddep_wait();       // the attention grid (and its memory) is complete
     const int tid = threadIdx.x;
     const int64_t r = blockIdx.x;
@@ -1888,7 +1940,8 @@ mla_status_t mla_decode_metadata(const int32_t *cache_seqlens, int B, int s_q, i
          reinterpret_cast<uintptr_t>(num_splits)) & 3)
         return MLA_ERR_MISALIGNED;
     const int tuples = num_sms / sh.G;
-    mla_metadata_kernel<<<1, kMetaThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+    const size_t smem = B <= 32 ? 32 * sizeof(int) : (2 * static_cast<size_t>(B + 1) + 33) * sizeof(int);
+    mla_metadata_kernel<<<1, kMetaThreads, smem, static_cast<cudaStream_t>(stream)>>>(
         cache_seqlens, B, s_q, H, num_sms, tuples, sh.G, sched_meta, num_splits);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "mla_metadata_kernel launch");
