@@ -86,24 +86,29 @@ constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
 constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
 constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
 constexpr int kBarDrainO = kBarDrain + 1;
-// FP8 cache (16 query columns): a ring of staging units between the TMA and
-// the bf16 chunk ring.  A unit is one 128-column group of the tile's 128 rows
-// in e4m3 (two 8 KB page halves, 128-byte swizzled), then, for a tile's first
-// unit, its 128 token scales; 17 KB keeps every unit 1024-byte aligned.
-constexpr int kF8Ring = 4;
+// FP8 cache (16 query columns), widened in place.  A ring slot (two bf16
+// chunks, 32 KB) first receives the e4m3 codes of its 128 columns of the
+// tile (128 rows x 128 bytes, both pages, 128-byte swizzled) in its upper
+// 16 KB; the converter warps then overwrite the slot row by row with the two
+// bf16 chunks (thread r reads its whole code row before writing its bf16
+// rows, and its code row is its own row of the upper chunk, so no thread
+// overwrites another's codes).  The tile's 128 token scales land in a ring of
+// 512-byte buffers after the slot ring.
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
-constexpr uint32_t kF8Unit = 17408;
-constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B
-constexpr uint32_t kF8ScaleOff = 16384;
-constexpr int kBarF8Full = kBarDrainO + 1;         // [kF8Ring] unit loaded
-constexpr int kBarF8Empty = kBarF8Full + kF8Ring;  // [kF8Ring] unit converted
-// FP8: the token scales of a tile, copied by the converter warps for the
-// softmax (a unit is handed back to the producer before the softmax runs).
+constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
+constexpr uint32_t kF8CodeOff = 16384;     // codes in the slot's upper half
+constexpr int kRawScBufs = 4;
+constexpr uint32_t kRawScBytes = kRawScBufs * 512;
+// The barrier block below keeps the layout of an earlier staging-ring design
+// (the bf16 instances are laid out exactly as before); the FP8 instance uses
+// its first kMaxF8Ring entries as per-slot "codes landed" barriers.
+constexpr int kBarF8Full = kBarDrainO + 1;
+constexpr int kBarRawFull = kBarF8Full;            // [ring slots] a slot's codes (and scales) landed
 constexpr int kScBufs = 4;
-constexpr uint32_t kScBytes = kScBufs * 128 * 4;
-constexpr int kBarScFull = kBarF8Empty + kF8Ring;  // [kScBufs] scales of a tile written
-constexpr int kBarScEmpty = kBarScFull + kScBufs;  // [kScBufs] scales read by the softmax
-constexpr int kNumBars = kBarScEmpty + kScBufs;
+constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // FP8: the softmax's copy of the token scales
+constexpr int kBarF8Reserved = kBarF8Full + 8 + 2 * kScBufs;
+constexpr int kMaxF8Ring = kBarF8Reserved - kBarRawFull;
+constexpr int kNumBars = kBarF8Reserved;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
 constexpr uint32_t kMiscRedOffset = (kNumBars * 8 + 127) / 128 * 128;
@@ -623,29 +628,30 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
             const int phys1 = __shfl_sync(0xffffffffu, cur, 2 * t + 1 - win);
             const bool live1 = (t * kTile + kPage) < L;
             if constexpr (F8) {
-                // FP8: the tile's five 128-column groups into the staging ring,
-                // the token scales with the first; the transposer warps turn
-                // each unit into one bf16 ring slot.
+                // FP8: the codes of the tile's five 128-column groups into the
+                // upper halves of its five ring slots, the token scales with the
+                // first; the converter warps widen each slot in place.
                 const uint32_t b8 = live1 ? 2 * kF8Half : kF8Half;
                 const uint32_t bsc = live1 ? 512u : 256u;
+                const uint32_t scb = sm.f8 + ((cc / kF8Units) % kRawScBufs) * 512u;
 #pragma unroll 1
                 for (int k = 0; k < kF8Units; ++k) {
                     const uint32_t u = cc + k;
-                    const int us = static_cast<int>(u % kF8Ring);
-                    if (!warp_wait(sm.bar(kBarF8Empty + us), ((u / kF8Ring) & 1) ^ 1, sm.abort_flag, p.err)) {
+                    const int slot = static_cast<int>(u % R);
+                    if (!warp_wait(sm.bar(kBarEmpty + slot), ((u / R) & 1) ^ 1, sm.abort_flag, p.err)) {
                         ok = false;
                         cc += k;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarF8Full + us), b8 + (k == 0 ? bsc : 0u));
+                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarRawFull + slot), b8 + (k == 0 ? bsc : 0u));
                     if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
-                    const uint32_t dst = sm.f8 + us * kF8Unit;
-                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarF8Full + us), 128 * k, 0, phys0);
-                    if (live1) ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarF8Full + us), 128 * k, 0, phys1);
+                    const uint32_t dst = sm.slot(slot) + kF8CodeOff;
+                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarRawFull + slot), 128 * k, 0, phys0);
+                    if (live1)
+                        ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarRawFull + slot), 128 * k, 0, phys1);
                     if (k == 0) {
-                        ptx::tma_load_2d_elect(dst + kF8ScaleOff, sc_map, sm.bar(kBarF8Full + us), 0, phys0);
-                        if (live1)
-                            ptx::tma_load_2d_elect(dst + kF8ScaleOff + 256, sc_map, sm.bar(kBarF8Full + us), 0, phys1);
+                        ptx::tma_load_2d_elect(scb, sc_map, sm.bar(kBarRawFull + slot), 0, phys0);
+                        if (live1) ptx::tma_load_2d_elect(scb + 256, sc_map, sm.bar(kBarRawFull + slot), 0, phys1);
                     }
                 }
                 if (ok) cc += kF8Units;
@@ -681,8 +687,8 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     }
     if (!ok) {
         // Let every load this warp issued land before the CTA exits.
-        const uint32_t RR = F8 ? static_cast<uint32_t>(kF8Ring) : R;
-        const int full0 = F8 ? kBarF8Full : kBarFull;
+        const uint32_t RR = R;
+        const int full0 = F8 ? kBarRawFull : kBarFull;
         const uint32_t first = cc > RR ? cc - RR : 0;
         for (uint32_t u = first; u < cc; ++u)
             warp_wait(sm.bar(full0 + static_cast<int>(u % RR)), (u / RR) & 1, sm.abort_flag, p.err, false);
@@ -958,12 +964,12 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     bool ok = true;
 
     // FP8 cache: these four warps, idle for most of a tile at 16 query
-    // columns, widen the tile's five e4m3 staging units into its five bf16
-    // ring slots (thread = token row r: 128 codes -> bf16, exactly, in the
-    // swizzled layout TMA gives bf16 chunks), one tile ahead of their own
-    // softmax, so the transposer warps only transpose.  The tile's token
-    // scales go to a small ring read by the softmax (Smem::tscale).
-    uint32_t c8 = 0, cc8 = 0;            // staging units / ring slot uses converted
+    // columns, widen each of the tile's five ring slots in place (thread =
+    // token row r: its 128 codes -> bf16, exactly, in the swizzled layout TMA
+    // gives bf16 chunks), one tile ahead of their own softmax, so the
+    // transposer warps only transpose.  The tile's token scales go to a small
+    // ring read by the softmax (Smem::tscale).
+    uint32_t cc8 = 0;                     // ring slot uses converted
     uint32_t nconv = 0, total_tiles = 0;  // tiles converted / tiles of this CTA
     bool conv_ok = true;
     if constexpr (F8) {
@@ -980,15 +986,14 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         const uint32_t sw = r & 7u;
 #pragma unroll 1
         for (int k = 0; k < kF8Units; ++k) {
-            const uint32_t u8 = c8 + k;
-            const int us = static_cast<int>(u8 % kF8Ring);
-            conv_ok = conv_ok && warp_wait(sm.bar(kBarF8Full + us), (u8 / kF8Ring) & 1, sm.abort_flag, p.err);
             const uint32_t su = cc8 + k;
             const int slot = static_cast<int>(su % R);
-            conv_ok = conv_ok && warp_wait(sm.bar(kBarEmpty + slot), ((su / R) & 1) ^ 1, sm.abort_flag, p.err);
+            conv_ok = conv_ok && warp_wait(sm.bar(kBarRawFull + slot), (su / R) & 1, sm.abort_flag, p.err);
             if (!conv_ok) continue;
-            const uint32_t src = sm.f8 + us * kF8Unit;
-            if (k == 0) sm.tscale[(nconv % kScBufs) * 128 + r] = ptx::ld_shared_f32(src + kF8ScaleOff + 4u * r);
+            const uint32_t src = sm.slot(slot) + kF8CodeOff;
+            if (k == 0)
+                sm.tscale[(nconv % kScBufs) * 128 + r] =
+                    ptx::ld_shared_f32(sm.f8 + (nconv % kRawScBufs) * 512u + 4u * r);
             const uint32_t dst = sm.slot(slot) + r * 128u;
             const int nlu = (k == kF8Units - 1) ? 4 : 8;  // the rope group is 64 columns
 #pragma unroll
@@ -1012,12 +1017,8 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(sm.bar(kBarFull + slot));
-                ptx::mbar_arrive(sm.bar(kBarF8Empty + us));
-            }
+            if (lane == 0) ptx::mbar_arrive(sm.bar(kBarFull + slot));
         }
-        c8 += kF8Units;
         cc8 += C::SPT;
         ++nconv;
         ptx::named_bar_sync(1, 128);  // the tile's token scales, from every warp, before any reads them
@@ -1244,7 +1245,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.slot_bytes = C::SLOT_BYTES;
     uint32_t off = p.ring * C::SLOT_BYTES;
     sm.f8 = base + off;
-    if constexpr (F8) off += kF8Ring * kF8Unit;
+    if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
     sm.p = sm.q + C::QBYTES;
     uint8_t *misc = gbase + off + C::QBYTES + C::PBYTES;
@@ -1264,13 +1265,18 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
             ptx::mbar_init(sm.bar(kBarFull + s), F8 ? 4 : 1);  // FP8: the four converter warps
             ptx::mbar_init(sm.bar(kBarEmpty + s), C::EMPTY_ARRIVALS);
         }
-        for (int i = 0; i < kF8Ring; ++i) {
-            ptx::mbar_init(sm.bar(kBarF8Full + i), 1);
-            ptx::mbar_init(sm.bar(kBarF8Empty + i), 4);
-        }
-        for (int i = 0; i < kScBufs; ++i) {
-            ptx::mbar_init(sm.bar(kBarScFull + i), 4);   // the four converter warps
-            ptx::mbar_init(sm.bar(kBarScEmpty + i), 4);  // the four softmax warps
+        if constexpr (F8) {
+            for (int s = 0; s < p.ring; ++s) ptx::mbar_init(sm.bar(kBarRawFull + s), 1);
+        } else {
+            // (unused by the bf16 instances; kept so their set-up is unchanged)
+            for (int i = 0; i < 4; ++i) {
+                ptx::mbar_init(sm.bar(kBarF8Full + i), 1);
+                ptx::mbar_init(sm.bar(kBarF8Full + 4 + i), 4);
+            }
+            for (int i = 0; i < kScBufs; ++i) {
+                ptx::mbar_init(sm.bar(kBarF8Full + 8 + i), 4);
+                ptx::mbar_init(sm.bar(kBarF8Full + 8 + kScBufs + i), 4);
+            }
         }
         ptx::mbar_init(sm.bar(kBarQFull), 1);
         ptx::mbar_init(sm.bar(kBarQEmpty), 1);
@@ -1631,9 +1637,10 @@ int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
     const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024 +
-                                       (F8 ? kF8Ring * kF8Unit + kScBytes : 0));
+                                       (F8 ? kRawScBytes + kScBytes : 0));
     int R = (smem_optin - fixed) / static_cast<int>(C::SLOT_BYTES);
     if (R > kMaxRing) R = kMaxRing;
+    if (F8 && R > kMaxF8Ring) R = kMaxF8Ring;  // one "codes landed" barrier per slot
     *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * C::SLOT_BYTES;
     return R;
 }
