@@ -86,28 +86,30 @@ constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
 constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
 constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
 constexpr int kBarDrainO = kBarDrain + 1;
-// FP8 cache (16 query columns), widened in place.  A ring slot (two bf16
-// chunks, 32 KB) first receives the e4m3 codes of its 128 columns of the
-// tile (128 rows x 128 bytes, both pages, 128-byte swizzled) in its upper
-// 16 KB; the converter warps then overwrite the slot row by row with the two
-// bf16 chunks (thread r reads its whole code row before writing its bf16
-// rows, and its code row is its own row of the upper chunk, so no thread
-// overwrites another's codes).  The tile's 128 token scales land in a ring of
-// 512-byte buffers after the slot ring.
+// FP8 cache (16 query columns).  The producer TMA-loads each 128-column group
+// of a tile ("unit": 128 rows x 128 bytes of e4m3 codes, both pages, 128-byte
+// swizzled) into a ring of kF8Stage 16 KB staging slots, the tile's 128 token
+// scales with its first unit into a ring of 512-byte buffers.  The softmax
+// warps widen each unit into a bf16 ring slot (two chunks, 32 KB) as soon as
+// its codes have landed and the slot is free, between their own softmax
+// tiles, so the loads of later tiles stay in flight while a tile is widened,
+// read by the score MMA and transposed.
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
 constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
-constexpr uint32_t kF8CodeOff = 16384;     // codes in the slot's upper half
+constexpr int kF8Stage = 6;                // staging slots
+constexpr uint32_t kF8StageBytes = 16384;  // one unit's codes
 constexpr int kRawScBufs = 4;
 constexpr uint32_t kRawScBytes = kRawScBufs * 512;
-// The barrier block below keeps the layout of an earlier staging-ring design
-// (the bf16 instances are laid out exactly as before); the FP8 instance uses
-// its first kMaxF8Ring entries as per-slot "codes landed" barriers.
+// The barrier block below keeps the layout of an earlier design (the bf16
+// instances are laid out exactly as before); the FP8 instance uses its first
+// 2 x kF8Stage entries: per staging slot "codes landed" and "codes read".
 constexpr int kBarF8Full = kBarDrainO + 1;
-constexpr int kBarRawFull = kBarF8Full;            // [ring slots] a slot's codes (and scales) landed
+constexpr int kBarRawFull = kBarF8Full;            // [kF8Stage] a unit's codes (and the tile's scales) landed
+constexpr int kBarRawEmpty = kBarF8Full + 8;       // [kF8Stage] the four converter warps have read them
 constexpr int kScBufs = 4;
 constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // FP8: the softmax's copy of the token scales
 constexpr int kBarF8Reserved = kBarF8Full + 8 + 2 * kScBufs;
-constexpr int kMaxF8Ring = kBarF8Reserved - kBarRawFull;
+static_assert(kF8Stage <= 8 && kBarRawEmpty + kF8Stage <= kBarF8Reserved, "FP8 staging barriers");
 constexpr int kNumBars = kBarF8Reserved;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
@@ -629,29 +631,29 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
             const bool live1 = (t * kTile + kPage) < L;
             if constexpr (F8) {
                 // FP8: the codes of the tile's five 128-column groups into the
-                // upper halves of its five ring slots, the token scales with the
-                // first; the converter warps widen each slot in place.
+                // staging ring, the token scales with the first.
                 const uint32_t b8 = live1 ? 2 * kF8Half : kF8Half;
                 const uint32_t bsc = live1 ? 512u : 256u;
                 const uint32_t scb = sm.f8 + ((cc / kF8Units) % kRawScBufs) * 512u;
+                const uint32_t stage0 = sm.f8 - kF8Stage * kF8StageBytes;
 #pragma unroll 1
                 for (int k = 0; k < kF8Units; ++k) {
                     const uint32_t u = cc + k;
-                    const int slot = static_cast<int>(u % R);
-                    if (!warp_wait(sm.bar(kBarEmpty + slot), ((u / R) & 1) ^ 1, sm.abort_flag, p.err)) {
+                    const int st = static_cast<int>(u % kF8Stage);
+                    if (!warp_wait(sm.bar(kBarRawEmpty + st), ((u / kF8Stage) & 1) ^ 1, sm.abort_flag, p.err)) {
                         ok = false;
                         cc += k;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarRawFull + slot), b8 + (k == 0 ? bsc : 0u));
+                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarRawFull + st), b8 + (k == 0 ? bsc : 0u));
                     if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
-                    const uint32_t dst = sm.slot(slot) + kF8CodeOff;
-                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarRawFull + slot), 128 * k, 0, phys0);
+                    const uint32_t dst = stage0 + st * kF8StageBytes;
+                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarRawFull + st), 128 * k, 0, phys0);
                     if (live1)
-                        ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarRawFull + slot), 128 * k, 0, phys1);
+                        ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarRawFull + st), 128 * k, 0, phys1);
                     if (k == 0) {
-                        ptx::tma_load_2d_elect(scb, sc_map, sm.bar(kBarRawFull + slot), 0, phys0);
-                        if (live1) ptx::tma_load_2d_elect(scb + 256, sc_map, sm.bar(kBarRawFull + slot), 0, phys1);
+                        ptx::tma_load_2d_elect(scb, sc_map, sm.bar(kBarRawFull + st), 0, phys0);
+                        if (live1) ptx::tma_load_2d_elect(scb + 256, sc_map, sm.bar(kBarRawFull + st), 0, phys1);
                     }
                 }
                 if (ok) cc += kF8Units;
@@ -687,7 +689,7 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     }
     if (!ok) {
         // Let every load this warp issued land before the CTA exits.
-        const uint32_t RR = R;
+        const uint32_t RR = F8 ? kF8Stage : R;
         const int full0 = F8 ? kBarRawFull : kBarFull;
         const uint32_t first = cc > RR ? cc - RR : 0;
         for (uint32_t u = first; u < cc; ++u)
@@ -964,64 +966,89 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     bool ok = true;
 
     // FP8 cache: these four warps, idle for most of a tile at 16 query
-    // columns, widen each of the tile's five ring slots in place (thread =
-    // token row r: its 128 codes -> bf16, exactly, in the swizzled layout TMA
-    // gives bf16 chunks), one tile ahead of their own softmax, so the
-    // transposer warps only transpose.  The tile's token scales go to a small
-    // ring read by the softmax (Smem::tscale).
-    uint32_t cc8 = 0;                     // ring slot uses converted
-    uint32_t nconv = 0, total_tiles = 0;  // tiles converted / tiles of this CTA
-    bool conv_ok = true;
+    // columns, also widen the staged codes into the bf16 ring, unit by unit
+    // (thread = token row r: its 128 codes -> bf16, exactly, in the swizzled
+    // layout TMA gives bf16 chunks), so the transposer warps only transpose.
+    // Each warp polls on its own: it runs its softmax of tile it as soon as
+    // S^T(it) is ready, and otherwise widens its 32 rows of the next unit
+    // whose codes have landed and whose ring slot is free.  Neither poll
+    // blocks, so no wait of this warp depends on a softmax it has not done.
+    // The tile's token scales go to a small ring read by the softmax
+    // (Smem::tscale); each warp reads only its own rows of it.
+    uint32_t cu8 = 0, total_units = 0;  // units widened by this warp / units of this CTA
     if constexpr (F8) {
         for (int b = w.b0; b <= w.b1; ++b) {
             const int nt = tiles_of(max(0, __ldg(p.seqlens + b)));
             const int tb = (b == w.b0) ? w.t0 : 0;
             const int te = min((b == w.b1) ? w.t1 : nt, nt);
-            total_tiles += static_cast<uint32_t>(max(0, te - tb));
+            total_units += static_cast<uint32_t>(max(0, te - tb)) * kF8Units;
         }
     }
-    auto convert_tile = [&]() {
+    auto convert_unit = [&]() -> bool {
+        if (cu8 >= total_units) return false;
         const uint32_t R = static_cast<uint32_t>(p.ring);
+        const int st = static_cast<int>(cu8 % kF8Stage);
+        const int slot = static_cast<int>(cu8 % R);
+        const bool rdy = ptx::mbar_test_wait(sm.bar(kBarRawFull + st), (cu8 / kF8Stage) & 1) &&
+                         ptx::mbar_test_wait(sm.bar(kBarEmpty + slot), ((cu8 / R) & 1) ^ 1);
+        if (!__all_sync(0xffffffffu, rdy)) return false;
         const uint32_t r = static_cast<uint32_t>(32 * wq + lane);
         const uint32_t sw = r & 7u;
-#pragma unroll 1
-        for (int k = 0; k < kF8Units; ++k) {
-            const uint32_t su = cc8 + k;
-            const int slot = static_cast<int>(su % R);
-            conv_ok = conv_ok && warp_wait(sm.bar(kBarRawFull + slot), (su / R) & 1, sm.abort_flag, p.err);
-            if (!conv_ok) continue;
-            const uint32_t src = sm.slot(slot) + kF8CodeOff;
-            if (k == 0)
-                sm.tscale[(nconv % kScBufs) * 128 + r] =
-                    ptx::ld_shared_f32(sm.f8 + (nconv % kRawScBufs) * 512u + 4u * r);
-            const uint32_t dst = sm.slot(slot) + r * 128u;
-            const int nlu = (k == kF8Units - 1) ? 4 : 8;  // the rope group is 64 columns
+        const uint32_t k = cu8 % kF8Units, tile = cu8 / kF8Units;
+        const uint32_t src = sm.f8 - kF8Stage * kF8StageBytes + st * kF8StageBytes + r * 128u;
+        if (k == 0)
+            sm.tscale[(tile % kScBufs) * 128 + r] = ptx::ld_shared_f32(sm.f8 + (tile % kRawScBufs) * 512u + 4u * r);
+        const uint32_t dst = sm.slot(slot) + r * 128u;
+        // The row's eight 16-byte groups are loaded before any is widened, so
+        // the loads overlap.  The rope group's upper 64 columns are the zero
+        // fill of its TMA box; widened, they land in the slot's second chunk,
+        // which nothing reads.
+        uint4 cw[8];
 #pragma unroll
-            for (int lu = 0; lu < 8; ++lu) {
-                if (lu < nlu) {
-                    const uint4 wv = ptx::ld_shared_v4(src + r * 128u + ((static_cast<uint32_t>(lu) ^ sw) << 4));
-                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-                    uint32_t o[8];
+        for (int lu = 0; lu < 8; ++lu) cw[lu] = ptx::ld_shared_v4(src + ((static_cast<uint32_t>(lu) ^ sw) << 4));
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 lo = ptx::e4m3x2_to_float2(words[i], false);
-                        const float2 hi = ptx::e4m3x2_to_float2(words[i], true);
-                        o[2 * i] = ptx::pack_bf16x2(lo.x, lo.y);  // exact: e4m3 values are bf16 values
-                        o[2 * i + 1] = ptx::pack_bf16x2(hi.x, hi.y);
+        for (int lu = 0; lu < 8; ++lu) {
+            const uint32_t words[4] = {cw[lu].x, cw[lu].y, cw[lu].z, cw[lu].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ptx::e4m3x4_to_bf16x4(words[i], o[2 * i], o[2 * i + 1]);
+            const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
+            const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
+            ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            ptx::mbar_arrive(sm.bar(kBarFull + slot));
+            ptx::mbar_arrive(sm.bar(kBarRawEmpty + st));
+        }
+        ++cu8;
+        return true;
+    };
+    // FP8: until S^T(it) is ready, widen what can be widened (bounded like
+    // wait_bounded; the outcome is warp-uniform).
+    auto poll_scores = [&](uint32_t sbar, uint32_t parity) -> bool {
+        uint64_t t0 = 0;
+        uint32_t idle = 0;
+        while (true) {
+            if (__all_sync(0xffffffffu, ptx::mbar_test_wait(sbar, parity))) return true;
+            if (convert_unit()) continue;
+            // nothing to widen: park on the scores for a moment (the issue
+            // slots go to the transposer warps of this sub-partition)
+            if (__all_sync(0xffffffffu, ptx::mbar_try_wait(sbar, parity, 200u))) return true;
+            if (idle++ == 0) t0 = ptx::globaltimer_ns();
+            if ((idle & 3u) == 0) {
+                if (__any_sync(0xffffffffu, *sm.abort_flag != 0)) return false;
+                if (__any_sync(0xffffffffu, ptx::globaltimer_ns() - t0 > kWaitLimitNs)) {
+                    if (lane == 0) {
+                        *sm.abort_flag = 1;
+                        atomicOr(p.err, MLA_DEVERR_TIMEOUT);
                     }
-                    const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
-                    const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
-                    ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
-                    ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                    return false;
                 }
             }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(sm.bar(kBarFull + slot));
         }
-        cc8 += C::SPT;
-        ++nconv;
-        ptx::named_bar_sync(1, 128);  // the tile's token scales, from every warp, before any reads them
     };
 
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
@@ -1038,13 +1065,11 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         bool wait_ok = true;  // a failed wait is carried to the next agreement point
 
         for (int t = tb; t < te; ++t) {
-            if constexpr (F8) {
-                // keep the converted tiles one ahead of this softmax (tile it + 1)
-                while (nconv < total_tiles && nconv <= it + 1) convert_tile();
-                wait_ok = wait_ok && conv_ok;
-            }
             const uint32_t sb = it % C::NS, su = it / C::NS;
-            wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
+            if constexpr (F8)
+                wait_ok = poll_scores(sm.bar(kBarSFull + sb), su & 1) && wait_ok;
+            else
+                wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
             ptx::tc_fence_after();
             uint32_t raw[2][4 * NG];
 #pragma unroll
@@ -1064,7 +1089,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             // past the visible tokens, so their zero weights stay zero)
             float tsc[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
             if constexpr (F8) {
-                const uint32_t sbuf = it % kScBufs;  // written by convert_tile, behind a named barrier
+                const uint32_t sbuf = it % kScBufs;  // written by this warp's convert_unit
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -1244,6 +1269,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.ring = base;
     sm.slot_bytes = C::SLOT_BYTES;
     uint32_t off = p.ring * C::SLOT_BYTES;
+    if constexpr (F8) off += kF8Stage * kF8StageBytes;  // FP8: the staging ring, then the token scales
     sm.f8 = base + off;
     if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
@@ -1266,7 +1292,10 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
             ptx::mbar_init(sm.bar(kBarEmpty + s), C::EMPTY_ARRIVALS);
         }
         if constexpr (F8) {
-            for (int s = 0; s < p.ring; ++s) ptx::mbar_init(sm.bar(kBarRawFull + s), 1);
+            for (int s = 0; s < kF8Stage; ++s) {
+                ptx::mbar_init(sm.bar(kBarRawFull + s), 1);
+                ptx::mbar_init(sm.bar(kBarRawEmpty + s), 4);
+            }
         } else {
             // (unused by the bf16 instances; kept so their set-up is unchanged)
             for (int i = 0; i < 4; ++i) {
@@ -1365,19 +1394,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
 
 // =============================================================== combine
 // One 128-thread block per output row (b, i, h) of a sequence cut into pieces.
-// Each thread owns four latent dims and issues the loads of a batch of 20
-// pieces together (the ~19 pieces of a 64K-context sequence split over 148
-// SMs in one memory round trip instead of three of 8).  Launched as a
+// Each thread owns four latent dims and issues the loads of a batch of
+// pieces together.  Two instances: 20 pieces per batch (128 registers, four
+// blocks per SM) when the rows fit in one wave -- the ~19 pieces of a
+// 64K-context sequence split over 148 SMs in one memory round trip -- and 8
+// pieces (64 registers, eight blocks per SM) for many rows of few pieces
+// (8192 rows at 128 heads), where resident blocks matter more.  Launched as a
 // programmatic dependent of the attention kernel: it may become resident
 // early and waits in hardware for that grid to finish.
 constexpr int kCombineThreads = 128;
 
-__global__ void __launch_bounds__(kCombineThreads, 4)
+template <int kBatch>
+__global__ void __launch_bounds__(kCombineThreads, kBatch > 8 ? 4 : 8)
 mla_combine_kernel(const int32_t *__restrict__ split_base, const float *__restrict__ ws_o,
                    const float *__restrict__ ws_lse, int B, int s_q, int H, int HG, int G, int max_pieces,
                    uint16_t *__restrict__ out, float *__restrict__ lse, int32_t *__restrict__ err)
 {
-    constexpr int kBatch = 20;  // pieces whose loads are in flight together
     ptx::griddep_wait();       // the attention grid (and its memory) is complete
     const int tid = threadIdx.x;
     const int64_t r = blockIdx.x;
@@ -1637,10 +1669,9 @@ int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
     const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024 +
-                                       (F8 ? kRawScBytes + kScBytes : 0));
+                                       (F8 ? kF8Stage * kF8StageBytes + kRawScBytes + kScBytes : 0));
     int R = (smem_optin - fixed) / static_cast<int>(C::SLOT_BYTES);
     if (R > kMaxRing) R = kMaxRing;
-    if (F8 && R > kMaxF8Ring) R = kMaxF8Ring;  // one "codes landed" barrier per slot
     *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * C::SLOT_BYTES;
     return R;
 }
@@ -1984,7 +2015,10 @@ mla_status_t mla_decode_combine(const int32_t *num_splits, const int32_t *sched_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mla_combine_kernel, num_splits, ws_o, ws_lse, B, s_q, H, sh.HG, sh.G,
+    // one wave of 4 blocks per SM (of num_sms SMs): the wide batch
+    const bool wide = rows <= 4ll * num_sms;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wide ? mla_combine_kernel<20> : mla_combine_kernel<8>, num_splits, ws_o,
+                                       ws_lse, B, s_q, H, sh.HG, sh.G,
                                        wl.pieces, out, lse, const_cast<int32_t *>(sched_meta));
     if (e != cudaSuccess) return cuda_fail(e, "mla_combine_kernel launch");
     return MLA_OK;

@@ -49,6 +49,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
     return ok != 0;
 }
 
+// True if the phase with the given parity has completed; returns at once
+// either way (no suspension), for loops that poll several barriers.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
 {
@@ -405,20 +420,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Two e4m3 values (bytes 0 and 1 of `x` when `high` is false, bytes 2 and 3
-// when true) to fp32, exactly: e4m3 -> f16 (every e4m3 value is an f16
-// value) -> f32.  Byte order is kept: f.x comes from the lower byte.
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t x, bool high)
+// Four e4m3 codes (the bytes of x, lowest first) -> four bf16 values, as two
+// bf16x2 words (codes 0, 1 in lo; 2, 3 in hi), exactly: e4m3 -> f16 (every
+// e4m3 value is an f16 value) -> f32 -> bf16 (and a bf16 value).  The NaN
+// codes stay NaN.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t &lo, uint32_t &hi)
 {
-    uint32_t h;
-    if (high)
-        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}" : "=r"(h) : "r"(x));
-    else
-        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h) : "r"(x));
-    float2 f;
-    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-        : "=f"(f.x), "=f"(f.y) : "r"(h));
-    return f;
+    uint32_t h0, h1;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(h0) : "r"(x));
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}" : "=r"(h1) : "r"(x));
+    float a0, a1, b0, b1;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(a0), "=f"(a1) : "r"(h0));
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(b0), "=f"(b1) : "r"(h1));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(a1), "f"(a0));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(b1), "f"(b0));
 }
 
 }  // namespace ptx

@@ -62,6 +62,27 @@ def test_fp8_tail_codes_never_reach_the_result(dev, orc):
     compare(g_out, g_lse, r_out, r_lse, what="fp8 NaN tails")
 
 
+def test_fp8_widening_is_exact_for_every_code(dev):
+    # One visible token with scale 1: its weight is 1, so each output row is
+    # the token's 512 value columns as widened by the kernel.  The row holds
+    # every code but the two NaN patterns s|1111|111, twice (subnormals and
+    # both zeros included), checked against torch's float8_e4m3fn decoding.
+    inp = mi.small(B=1, s_q=1, H=16, seqlens=[1], seed=68)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=69)
+    finite = torch.tensor([c for c in range(256) if c & 0x7F != 0x7F] + [0x38, 0xB8])
+    codes = torch.cat([finite, finite.flip(0), torch.full((64,), 0x38)]).to(torch.uint8)
+    assert codes.numel() == 576
+    blk = int(inp.block_table[0, 0])
+    cache.codes[blk, 0] = codes
+    cache.scale[blk, 0] = 1.0
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err == 0 and np.all(np.isfinite(g_lse))
+    expect = codes[:512].view(torch.float8_e4m3fn).float().numpy()
+    assert np.all(np.isfinite(expect))
+    for h in range(16):
+        np.testing.assert_array_equal(g_out[0, 0, h], expect)
+
+
 def test_fp8_paging_invariance(dev):
     # the same logical rows through an identity and a shuffled table: bitwise equal
     a = mi.small(B=2, s_q=1, H=16, seqlens=[300, 900], table="identity", seed=64)
