@@ -86,30 +86,39 @@ constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
 constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
 constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
 constexpr int kBarDrainO = kBarDrain + 1;
-// FP8 cache (16 query columns).  The producer TMA-loads each 128-column group
-// of a tile ("unit": 128 rows x 128 bytes of e4m3 codes, both pages, 128-byte
-// swizzled) into a ring of kF8Stage 16 KB staging slots, the tile's 128 token
-// scales with its first unit into a ring of 512-byte buffers.  The softmax
-// warps widen each unit into a bf16 ring slot (two chunks, 32 KB) as soon as
-// its codes have landed and the slot is free, between their own softmax
-// tiles, so the loads of later tiles stay in flight while a tile is widened,
-// read by the score MMA and transposed.
+// FP8 cache (16 query columns).  The tensor cores read the e4m3 codes as
+// they lie in the cache (tcgen05.mma kind::f8f6f4): the ring's slots are 16 KB
+// "units", one 128-column group of a tile (128 rows x 128 bytes of codes, both
+// pages, 128-byte swizzled), five per tile, the last holding the 64 rope
+// columns and the zero fill of its TMA box.  The score MMA reads a unit
+// K-major (rows = tokens); the output MMA reads latent units 0-3 again,
+// MN-major (rows = tokens, the 128 latent dims contiguous), as V^T.  The
+// tile's 128 token scales land with its first unit in a ring of 512-byte
+// buffers after the slot ring.
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
 constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
-constexpr int kF8Stage = 6;                // staging slots
-constexpr uint32_t kF8StageBytes = 16384;  // one unit's codes
+constexpr uint32_t kF8UnitBytes = 16384;   // one ring slot: a unit's codes
 constexpr int kRawScBufs = 4;
 constexpr uint32_t kRawScBytes = kRawScBufs * 512;
+// q split into two e4m3 terms per element (see softmax_warps), per unit a hi
+// and a lo tile of 16 rows x 128 B, 128-byte swizzled, K-major.
+constexpr uint32_t kQsUnitBytes = 4096;
+constexpr uint32_t kQsBytes = kF8Units * kQsUnitBytes;
+// FP8 weights: the reference max sits kLift8 below the largest log2 weight
+// seen when it last moved, so weights reach 2^kLift8 and stay above e4m3's
+// subnormal range (2^-6) down to 2^-13 of the largest; it moves again when a
+// weight would pass 2^kTau8 (e4m3 holds up to 448).  l and lse use the same
+// reference, so the result does not depend on it.
+constexpr float kLift8 = 7.f;
+constexpr float kTau8 = 8.f;
 // The barrier block below keeps the layout of an earlier design (the bf16
 // instances are laid out exactly as before); the FP8 instance uses its first
-// 2 x kF8Stage entries: per staging slot "codes landed" and "codes read".
+// entry for "q split written".
 constexpr int kBarF8Full = kBarDrainO + 1;
-constexpr int kBarRawFull = kBarF8Full;            // [kF8Stage] a unit's codes (and the tile's scales) landed
-constexpr int kBarRawEmpty = kBarF8Full + 8;       // [kF8Stage] the four converter warps have read them
+constexpr int kBarQsFull = kBarF8Full;
 constexpr int kScBufs = 4;
-constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // FP8: the softmax's copy of the token scales
+constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // FP8: per-row q scales (first 16 words)
 constexpr int kBarF8Reserved = kBarF8Full + 8 + 2 * kScBufs;
-static_assert(kF8Stage <= 8 && kBarRawEmpty + kF8Stage <= kBarF8Reserved, "FP8 staging barriers");
 constexpr int kNumBars = kBarF8Reserved;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
@@ -589,7 +598,7 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     using C = Cfg<N, SQ>;
     const int lane = threadIdx.x & 31;
     const uint32_t R = static_cast<uint32_t>(p.ring);
-    uint32_t cc = 0;  // ring slot uses so far (bf16 cache) / staging unit uses so far (FP8 cache)
+    uint32_t cc = 0;  // ring slot uses so far (FP8 cache: one per unit)
     int qi = 0;       // Q loads so far
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
@@ -630,30 +639,29 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
             const int phys1 = __shfl_sync(0xffffffffu, cur, 2 * t + 1 - win);
             const bool live1 = (t * kTile + kPage) < L;
             if constexpr (F8) {
-                // FP8: the codes of the tile's five 128-column groups into the
-                // staging ring, the token scales with the first.
+                // FP8: the codes of the tile's five 128-column groups, one ring
+                // slot each, the token scales with the first.
                 const uint32_t b8 = live1 ? 2 * kF8Half : kF8Half;
                 const uint32_t bsc = live1 ? 512u : 256u;
                 const uint32_t scb = sm.f8 + ((cc / kF8Units) % kRawScBufs) * 512u;
-                const uint32_t stage0 = sm.f8 - kF8Stage * kF8StageBytes;
 #pragma unroll 1
                 for (int k = 0; k < kF8Units; ++k) {
                     const uint32_t u = cc + k;
-                    const int st = static_cast<int>(u % kF8Stage);
-                    if (!warp_wait(sm.bar(kBarRawEmpty + st), ((u / kF8Stage) & 1) ^ 1, sm.abort_flag, p.err)) {
+                    const int slot = static_cast<int>(u % R);
+                    if (!warp_wait(sm.bar(kBarEmpty + slot), ((u / R) & 1) ^ 1, sm.abort_flag, p.err)) {
                         ok = false;
                         cc += k;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarRawFull + st), b8 + (k == 0 ? bsc : 0u));
+                    ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarFull + slot), b8 + (k == 0 ? bsc : 0u));
                     if (u == 0 && static_cast<int>(blockIdx.x) == p.debug_stall_cta) continue;
-                    const uint32_t dst = stage0 + st * kF8StageBytes;
-                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarRawFull + st), 128 * k, 0, phys0);
+                    const uint32_t dst = sm.slot(slot);
+                    ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarFull + slot), 128 * k, 0, phys0);
                     if (live1)
-                        ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarRawFull + st), 128 * k, 0, phys1);
+                        ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarFull + slot), 128 * k, 0, phys1);
                     if (k == 0) {
-                        ptx::tma_load_2d_elect(scb, sc_map, sm.bar(kBarRawFull + st), 0, phys0);
-                        if (live1) ptx::tma_load_2d_elect(scb + 256, sc_map, sm.bar(kBarRawFull + st), 0, phys1);
+                        ptx::tma_load_2d_elect(scb, sc_map, sm.bar(kBarFull + slot), 0, phys0);
+                        if (live1) ptx::tma_load_2d_elect(scb + 256, sc_map, sm.bar(kBarFull + slot), 0, phys1);
                     }
                 }
                 if (ok) cc += kF8Units;
@@ -689,8 +697,8 @@ __device__ void producer_warp(const DecodeParams &p, const Range &w, int g, cons
     }
     if (!ok) {
         // Let every load this warp issued land before the CTA exits.
-        const uint32_t RR = F8 ? kF8Stage : R;
-        const int full0 = F8 ? kBarRawFull : kBarFull;
+        const uint32_t RR = R;
+        const int full0 = kBarFull;
         const uint32_t first = cc > RR ? cc - RR : 0;
         for (uint32_t u = first; u < cc; ++u)
             warp_wait(sm.bar(full0 + static_cast<int>(u % RR)), (u / RR) & 1, sm.abort_flag, p.err, false);
@@ -801,6 +809,114 @@ __device__ void output_mma_warp(const DecodeParams &p, const Range &w, const Sme
     warp_wait(sm.bar(kBarDrainO), 0, sm.abort_flag, p.err, false);
 }
 
+// -- FP8 cache: the two MMA warps on the e4m3 codes ------------------------
+// Score MMA: S^T(t) = sum over the tile's five units of K_unit q_unit^T, with
+// q as its two e4m3 terms (hi, lo), K = 32 codes per instruction.  Latent
+// units stay in the ring for the output MMA; the rope unit is free after the
+// score MMA (both of its slot's arrivals come from here).
+template <int N, int SQ>
+__device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
+{
+    using C = Cfg<N, SQ>;
+    constexpr uint32_t idS = ptx::idesc_e4m3_f32(128, N, false, false);  // codes K-major, q terms K-major
+    const uint32_t R = static_cast<uint32_t>(p.ring);
+    const uint32_t qs = sm.f8 - kQsBytes;
+    uint32_t cc = 0, it = 0;
+    int qi = 0;
+    bool ok = true;
+    for (int b = w.b0; b <= w.b1 && ok; ++b) {
+        const int L = max(0, __ldg(p.seqlens + b));
+        const int nt = tiles_of(L);
+        const int tb = (b == w.b0) ? w.t0 : 0;
+        const int te = min((b == w.b1) ? w.t1 : nt, nt);
+        if (tb >= te) continue;
+        if (!(ok = warp_wait(sm.bar(kBarQsFull), qi & 1, sm.abort_flag, p.err))) break;
+        ++qi;
+        ptx::tc_fence_after();
+        for (int t = tb; t < te && ok; ++t) {
+            const uint32_t sb = it % C::NS, su = it / C::NS;
+            if (su >= 1 && !(ok = warp_wait(sm.bar(kBarSEmpty + sb), (su & 1) ^ 1, sm.abort_flag, p.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t d = tmem + C::S_COL + sb * N;
+#pragma unroll 1
+            for (int k = 0; k < kF8Units; ++k) {
+                const uint32_t u = cc + k;
+                const int slot = static_cast<int>(u % R);
+                if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
+                ptx::tc_fence_after();
+                const uint32_t a0 = sm.slot(slot);
+                const uint32_t q0 = qs + k * kQsUnitBytes;
+                const int steps = (k == kF8Units - 1) ? 2 : 4;  // the rope unit: 64 columns
+#pragma unroll 1
+                for (int kk = 0; kk < steps; ++kk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        ptx::mma_e4m3_ss_elect(d, ptx::desc_sw128(a0 + 32u * kk, 16, 1024),
+                                               ptx::desc_sw128(q0 + h * 2048u + 32u * kk, 16, 1024), idS,
+                                               (k | kk | h) != 0);
+                ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+                if (k == kF8Units - 1) ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+            }
+            if (!ok) break;
+            ptx::mma_commit_elect(sm.bar(kBarSFull + sb));
+            if (t == te - 1) ptx::mma_commit_elect(sm.bar(kBarQEmpty));
+            cc += kF8Units;
+            ++it;
+        }
+    }
+    ptx::mma_commit_elect(sm.bar(kBarDrain));
+    warp_wait(sm.bar(kBarDrain), 0, sm.abort_flag, p.err, false);
+}
+
+// Output MMA: O^T block j += V^T_j P~^T, V^T_j = latent unit j of the tile read
+// MN-major straight from its ring slot, P~ the weights as two e4m3 terms (hi,
+// lo: N rows x 128 tokens each, K-major), 32 tokens per instruction.  Each
+// unit's slot is free once its MMAs are complete.
+template <int N, int SQ>
+__device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
+{
+    using C = Cfg<N, SQ>;
+    constexpr uint32_t idO = ptx::idesc_e4m3_f32(128, N, true, false);  // V^T MN-major, P~^T K-major
+    const uint32_t R = static_cast<uint32_t>(p.ring);
+    uint32_t it = 0, cc = 0;
+    bool ok = true;
+    for (int b = w.b0; b <= w.b1 && ok; ++b) {
+        const int L = max(0, __ldg(p.seqlens + b));
+        const int nt = tiles_of(L);
+        const int tb = (b == w.b0) ? w.t0 : 0;
+        const int te = min((b == w.b1) ? w.t1 : nt, nt);
+        for (int t = tb; t < te && ok; ++t) {
+            const uint32_t pb = it & 1, pu = it >> 1;
+            if (!(ok = warp_wait(sm.bar(kBarPFull + pb), pu & 1, sm.abort_flag, p.err))) break;
+            ptx::tc_fence_after();
+            const uint32_t pa = sm.p + pb * 2 * C::QCHUNK;
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t u = cc + j;
+                const int slot = static_cast<int>(u % R);
+                // landed long ago (the score MMA read it); waited on for the ordering
+                if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
+                ptx::tc_fence_after();
+                const uint32_t a0 = sm.slot(slot);
+#pragma unroll 1
+                for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        ptx::mma_e4m3_ss_elect(tmem + j * N, ptx::desc_sw128(a0 + 4096u * kk, 8192, 1024),
+                                               ptx::desc_sw128(pa + h * 2048u + 32u * kk, 16, 1024), idO,
+                                               (t != tb) || kk != 0 || h != 0);
+                ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+            }
+            if (!ok) break;
+            ptx::mma_commit_elect(sm.bar(kBarPEmpty + pb));
+            cc += kF8Units;
+            ++it;
+        }
+    }
+    ptx::mma_commit_elect(sm.bar(kBarDrainO));
+    warp_wait(sm.bar(kBarDrainO), 0, sm.abort_flag, p.err, false);
+}
+
 // -- transposer: 4 warps copy V(t) into the TMEM ring as V^T ----------------
 // Warp q owns TMEM lanes 32q..32q+31, i.e. latent dims 128j + 32q + (0..31)
 // of every 128-dim block j: half of chunk 2j + q/2.  Per 16 dims x 16 tokens
@@ -810,7 +926,7 @@ __device__ void transposer_warps(const DecodeParams &p, const Range &w, const Sm
 {
     using C = Cfg<N, SQ>;
     constexpr uint32_t NVT = C::NVT;
-    static_assert(!F8 || C::CPS == 2, "FP8 staging unit = one 2-chunk ring slot");
+    if constexpr (F8) return;  // the FP8 output MMA reads V^T from the ring
     const uint32_t R = static_cast<uint32_t>(p.ring);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;
@@ -965,90 +1081,88 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     uint32_t it = 0;   // tiles processed
     bool ok = true;
 
-    // FP8 cache: these four warps, idle for most of a tile at 16 query
-    // columns, also widen the staged codes into the bf16 ring, unit by unit
-    // (thread = token row r: its 128 codes -> bf16, exactly, in the swizzled
-    // layout TMA gives bf16 chunks), so the transposer warps only transpose.
-    // Each warp polls on its own: it runs its softmax of tile it as soon as
-    // S^T(it) is ready, and otherwise widens its 32 rows of the next unit
-    // whose codes have landed and whose ring slot is free.  Neither poll
-    // blocks, so no wait of this warp depends on a softmax it has not done.
-    // The tile's token scales go to a small ring read by the softmax
-    // (Smem::tscale); each warp reads only its own rows of it.
-    uint32_t cu8 = 0, total_units = 0;  // units widened by this warp / units of this CTA
-    if constexpr (F8) {
-        for (int b = w.b0; b <= w.b1; ++b) {
-            const int nt = tiles_of(max(0, __ldg(p.seqlens + b)));
-            const int tb = (b == w.b0) ? w.t0 : 0;
-            const int te = min((b == w.b1) ? w.t1 : nt, nt);
-            total_units += static_cast<uint32_t>(max(0, te - tb)) * kF8Units;
-        }
-    }
-    auto convert_unit = [&]() -> bool {
-        if (cu8 >= total_units) return false;
-        const uint32_t R = static_cast<uint32_t>(p.ring);
-        const int st = static_cast<int>(cu8 % kF8Stage);
-        const int slot = static_cast<int>(cu8 % R);
-        const bool rdy = ptx::mbar_test_wait(sm.bar(kBarRawFull + st), (cu8 / kF8Stage) & 1) &&
-                         ptx::mbar_test_wait(sm.bar(kBarEmpty + slot), ((cu8 / R) & 1) ^ 1);
-        if (!__all_sync(0xffffffffu, rdy)) return false;
-        const uint32_t r = static_cast<uint32_t>(32 * wq + lane);
-        const uint32_t sw = r & 7u;
-        const uint32_t k = cu8 % kF8Units, tile = cu8 / kF8Units;
-        const uint32_t src = sm.f8 - kF8Stage * kF8StageBytes + st * kF8StageBytes + r * 128u;
-        if (k == 0)
-            sm.tscale[(tile % kScBufs) * 128 + r] = ptx::ld_shared_f32(sm.f8 + (tile % kRawScBufs) * 512u + 4u * r);
-        const uint32_t dst = sm.slot(slot) + r * 128u;
-        // The row's eight 16-byte groups are loaded before any is widened, so
-        // the loads overlap.  The rope group's upper 64 columns are the zero
-        // fill of its TMA box; widened, they land in the slot's second chunk,
-        // which nothing reads.
-        uint4 cw[8];
+    // FP8 cache: at the start of each range these warps write q as two e4m3
+    // terms for the score MMA.  Row n of q (576 bf16 values, 8 significant
+    // bits each) is scaled by a power of two 2^a_n that puts its largest
+    // magnitude in [128, 256), then hi = e4m3(x) and lo = e4m3(x - hi): x - hi
+    // has at most four significant bits, so hi + lo = x exactly unless lo
+    // falls below the e4m3 normal range (|x| < 2^-2, i.e. 2^-10 of the row's
+    // largest value), where lo keeps its bits down to 2^-9.  The score
+    // columns are multiplied back by 2^-a_n (Smem::tscale[n]).  Thread: row
+    // n = stid / 8 and the 16-column groups stid % 8 + 8 i, i < 5 (groups
+    // 36-39 are the zero fill past column 575 that the rope unit's upper
+    // half meets).
+    uint32_t qsplits = 0;
+    auto split_q = [&]() -> bool {
+        const bool okq = wait_bounded(sm.bar(kBarQFull), qsplits & 1, sm.abort_flag, p.err);
+        ++qsplits;
+        const int n = stid >> 3, part = stid & 7;
+        const uint32_t qs = sm.f8 - kQsBytes;
+        auto load16 = [&](int gq, float (&v)[16]) {
+            const int c = gq >> 2, u0 = (gq & 3) * 2;
+            const uint32_t rowa = sm.q + c * C::QCHUNK + n * 128u;
 #pragma unroll
-        for (int lu = 0; lu < 8; ++lu) cw[lu] = ptx::ld_shared_v4(src + ((static_cast<uint32_t>(lu) ^ sw) << 4));
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint4 x = ptx::ld_shared_v4(rowa + ((static_cast<uint32_t>(u0 + hh) ^ (n & 7)) << 4));
+                const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int lu = 0; lu < 8; ++lu) {
-            const uint32_t words[4] = {cw[lu].x, cw[lu].y, cw[lu].z, cw[lu].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) ptx::e4m3x4_to_bf16x4(words[i], o[2 * i], o[2 * i + 1]);
-            const uint32_t cb = dst + (static_cast<uint32_t>(lu) >> 2) * kChunkBytes;
-            const uint32_t bu = (static_cast<uint32_t>(lu) & 3u) * 2u;
-            ptx::st_shared_v4(cb + ((bu ^ sw) << 4), o[0], o[1], o[2], o[3]);
-            ptx::st_shared_v4(cb + (((bu + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            ptx::mbar_arrive(sm.bar(kBarFull + slot));
-            ptx::mbar_arrive(sm.bar(kBarRawEmpty + st));
-        }
-        ++cu8;
-        return true;
-    };
-    // FP8: until S^T(it) is ready, widen what can be widened (bounded like
-    // wait_bounded; the outcome is warp-uniform).
-    auto poll_scores = [&](uint32_t sbar, uint32_t parity) -> bool {
-        uint64_t t0 = 0;
-        uint32_t idle = 0;
-        while (true) {
-            if (__all_sync(0xffffffffu, ptx::mbar_test_wait(sbar, parity))) return true;
-            if (convert_unit()) continue;
-            // nothing to widen: park on the scores for a moment (the issue
-            // slots go to the transposer warps of this sub-partition)
-            if (__all_sync(0xffffffffu, ptx::mbar_try_wait(sbar, parity, 200u))) return true;
-            if (idle++ == 0) t0 = ptx::globaltimer_ns();
-            if ((idle & 3u) == 0) {
-                if (__any_sync(0xffffffffu, *sm.abort_flag != 0)) return false;
-                if (__any_sync(0xffffffffu, ptx::globaltimer_ns() - t0 > kWaitLimitNs)) {
-                    if (lane == 0) {
-                        *sm.abort_flag = 1;
-                        atomicOr(p.err, MLA_DEVERR_TIMEOUT);
-                    }
-                    return false;
+                for (int e = 0; e < 4; ++e) {
+                    v[8 * hh + 2 * e] = __uint_as_float(wv[e] << 16);
+                    v[8 * hh + 2 * e + 1] = __uint_as_float(wv[e] & 0xFFFF0000u);
                 }
             }
+        };
+        float mx = 0.f;
+#pragma unroll 1
+        for (int i = 0; i < 5; ++i) {
+            const int gq = part + 8 * i;
+            if (gq >= 36) continue;
+            float v[16];
+            load16(gq, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
         }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        int ex = 0;
+        frexpf(mx, &ex);  // mx < 2^ex
+        const float up = ldexpf(1.f, 8 - ex);
+#pragma unroll 1
+        for (int i = 0; i < 5; ++i) {
+            const int gq = part + 8 * i;
+            float v[16];
+            if (gq < 36) {
+                load16(gq, v);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            }
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+                uint32_t hb[2], lb[2];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const float x0 = v[4 * e4 + 2 * e2] * up, x1 = v[4 * e4 + 2 * e2 + 1] * up;
+                    hb[e2] = ptx::f32x2_to_e4m3x2(x0, x1);
+                    float h0, h1;
+                    ptx::e4m3x2_to_f32x2(hb[e2], h0, h1);
+                    lb[e2] = ptx::f32x2_to_e4m3x2(x0 - h0, x1 - h1);
+                }
+                hw[e4] = hb[0] | (hb[1] << 16);
+                lw[e4] = lb[0] | (lb[1] << 16);
+            }
+            const uint32_t at = qs + (gq >> 3) * kQsUnitBytes + n * 128u +
+                                ((static_cast<uint32_t>(gq & 7) ^ static_cast<uint32_t>(n & 7)) << 4);
+            ptx::st_shared_v4(at, hw[0], hw[1], hw[2], hw[3]);
+            ptx::st_shared_v4(at + 2048u, lw[0], lw[1], lw[2], lw[3]);
+        }
+        if (part == 0) sm.tscale[n] = ldexpf(1.f, ex - 8);
+        ptx::fence_proxy_async_smem();
+        ptx::named_bar_sync(1, 128);
+        if (lane == 0) ptx::mbar_arrive(sm.bar(kBarQsFull));
+        return okq;
     };
 
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
@@ -1063,13 +1177,19 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) l[gi][0] = l[gi][1] = mu[gi][0] = mu[gi][1] = 0.f;
         bool wait_ok = true;  // a failed wait is carried to the next agreement point
+        float qsc[NG][2];     // FP8: 2^-a of this thread's columns
+        if constexpr (F8) {
+            wait_ok = split_q() && wait_ok;
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) {
+                qsc[gi][0] = sm.tscale[8 * gi + c2];
+                qsc[gi][1] = sm.tscale[8 * gi + c2 + 1];
+            }
+        }
 
         for (int t = tb; t < te; ++t) {
             const uint32_t sb = it % C::NS, su = it / C::NS;
-            if constexpr (F8)
-                wait_ok = poll_scores(sm.bar(kBarSFull + sb), su & 1) && wait_ok;
-            else
-                wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
+            wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
             ptx::tc_fence_after();
             uint32_t raw[2][4 * NG];
 #pragma unroll
@@ -1086,16 +1206,25 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             const bool first = (t == tb);
             const int tok0 = t * kTile + 32 * wq + r8;
             // FP8 cache: the scales of this thread's four token rows (0 for rows
-            // past the visible tokens, so their zero weights stay zero)
-            float tsc[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
+            // past the visible tokens), from the buffer that landed with the
+            // tile's first unit (which the score MMA waited for).  A token's
+            // weight in O is 2^(x - mu) tsc with x its log2-domain score;
+            // the reference max mu follows x + log2|tsc|, so that weight is
+            // at most 2^kTau8 in magnitude.  lgt = log2|tsc| (0 where tsc is 0)
+            // and sgt = the sign of tsc (0 where tsc is 0).
+            float tsc[2][2] = {{1.f, 1.f}, {1.f, 1.f}}, lgt[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            float sgt[2][2] = {{1.f, 1.f}, {1.f, 1.f}};
             if constexpr (F8) {
-                const uint32_t sbuf = it % kScBufs;  // written by this warp's convert_unit
+                const uint32_t sbuf = sm.f8 + (it % kRawScBufs) * 512u;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const int row = 32 * wq + r8 + 16 * hf + 8 * jj;
-                        tsc[hf][jj] = (tok0 + 16 * hf + 8 * jj < nvis0) ? sm.tscale[sbuf * 128 + row] : 0.f;
+                        const float x = (tok0 + 16 * hf + 8 * jj < nvis0) ? ptx::ld_shared_f32(sbuf + 4u * row) : 0.f;
+                        tsc[hf][jj] = x;
+                        lgt[hf][jj] = x != 0.f ? __log2f(fabsf(x)) : 0.f;
+                        sgt[hf][jj] = x > 0.f ? 1.f : (x < 0.f ? -1.f : 0.f);
                     }
             }
             float d[2][NG][4];
@@ -1113,9 +1242,14 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                         const int qi = (8 * gi) / HG;
                         const bool vis = tok < nvis0 + qi;
                         float s = __uint_as_float(raw[hf][4 * gi + j]);
-                        if constexpr (F8) s *= tsc[hf][j >> 1];
-                        d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, -mu[gi][j & 1]) : NEG_INF;
-                        flag = flag || (d[hf][gi][j] > kTau);
+                        if constexpr (F8) {
+                            s *= tsc[hf][j >> 1] * qsc[gi][j & 1];
+                            d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, lgt[hf][j >> 1] - mu[gi][j & 1]) : NEG_INF;
+                            flag = flag || (d[hf][gi][j] > kTau8);
+                        } else {
+                            d[hf][gi][j] = vis ? fmaf(s, p.scale_log2, -mu[gi][j & 1]) : NEG_INF;
+                            flag = flag || (d[hf][gi][j] > kTau);
+                        }
                     }
             __syncwarp();
             if (ptx::named_bar_or(1, 128, flag)) {
@@ -1145,7 +1279,11 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                 if (stid < N) {
                     const int n = stid;
                     const float x = fmaxf(fmaxf(sm.red[n], sm.red[N + n]), fmaxf(sm.red[2 * N + n], sm.red[3 * N + n]));
-                    const float sh = first ? (x == NEG_INF ? 0.f : x) : fmaxf(x, 0.f);
+                    float sh;
+                    if constexpr (F8)  // FP8: the tile's largest weight becomes 2^kLift8 (see kLift8)
+                        sh = first ? (x == NEG_INF ? 0.f : x - kLift8) : fmaxf(x - kLift8, 0.f);
+                    else
+                        sh = first ? (x == NEG_INF ? 0.f : x) : fmaxf(x, 0.f);
                     sm.shift[n] = sh;
                     sm.mu[n] = (first ? 0.f : sm.mu[n]) + sh;
                 }
@@ -1205,34 +1343,80 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                 wait_ok = wait_bounded(sm.bar(kBarPEmpty + (it & 1)), ((it >> 1) & 1) ^ 1, sm.abort_flag, p.err) &&
                           wait_ok;
             const uint32_t pbuf = sm.p + (it & 1) * 2 * C::QCHUNK;
+            if constexpr (F8) {
+                // FP8: l takes 2^(x - mu); O takes w = 2^(x - mu) tsc as two
+                // e4m3 terms, hi = e4m3(w) and lo = e4m3(w - hi) (8 significant
+                // bits together, like bf16), written as P~^T (row n, token k at
+                // n * 128 + ((k / 16) ^ (n % 8)) * 16 + k % 16; hi at pbuf, lo
+                // 2 KB after it)
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[NG][2];
+                for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                for (int gi = 0; gi < NG; ++gi) {
-                    const float p0 = ptx::ex2_approx(d[hf][gi][0]);  // masked entries: 2^-inf = 0
-                    const float p1 = ptx::ex2_approx(d[hf][gi][1]);
-                    const float p2 = ptx::ex2_approx(d[hf][gi][2]);
-                    const float p3 = ptx::ex2_approx(d[hf][gi][3]);
-                    l[gi][0] += p0 + p2;
-                    l[gi][1] += p1 + p3;
-                    if constexpr (F8) {  // V holds the codes: the token's scale goes with its weight
-                        pk[gi][0] = ptx::pack_bf16x2(p0 * tsc[hf][0], p1 * tsc[hf][0]);
-                        pk[gi][1] = ptx::pack_bf16x2(p2 * tsc[hf][1], p3 * tsc[hf][1]);
-                    } else {
+                    for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+                        for (int jh = 0; jh < 2; ++jh) {  // token row r8 + 16 hf + 8 jh, columns n, n + 1
+                            const float dl = d[hf][gi][2 * jh], dr = d[hf][gi][2 * jh + 1];
+                            l[gi][0] += ptx::ex2_approx(dl - lgt[hf][jh]);
+                            l[gi][1] += ptx::ex2_approx(dr - lgt[hf][jh]);
+                            const float w0 = ptx::ex2_approx(dl) * sgt[hf][jh];
+                            const float w1 = ptx::ex2_approx(dr) * sgt[hf][jh];
+                            const uint32_t hb = ptx::f32x2_to_e4m3x2(w0, w1);
+                            float h0, h1;
+                            ptx::e4m3x2_to_f32x2(hb, h0, h1);
+                            const uint32_t lb = ptx::f32x2_to_e4m3x2(w0 - h0, w1 - h1);
+                            const int k = 32 * wq + r8 + 16 * hf + 8 * jh;
+                            const int n = 8 * gi + c2;
+                            const uint32_t a0 = pbuf + n * 128u +
+                                                ((static_cast<uint32_t>(k >> 4) ^ static_cast<uint32_t>(n & 7)) << 4) +
+                                                static_cast<uint32_t>(k & 15);
+                            const uint32_t a1 = pbuf + (n + 1) * 128u +
+                                                ((static_cast<uint32_t>(k >> 4) ^ static_cast<uint32_t>((n + 1) & 7)) << 4) +
+                                                static_cast<uint32_t>(k & 15);
+                            ptx::st_shared_u8(a0, hb & 0xFFu);
+                            ptx::st_shared_u8(a1, hb >> 8);
+                            ptx::st_shared_u8(a0 + 2048u, lb & 0xFFu);
+                            ptx::st_shared_u8(a1 + 2048u, lb >> 8);
+                        }
+                // Rows past the sequence's end in its last tile hold whatever the
+                // cache (or an earlier unit) left there, NaN codes included; their
+                // weights are zero, and the V^T the output MMA reads must be finite
+                // too: this thread zeroes its row of the tile's four latent units.
+                const int valid = L - t * kTile;
+                const int r = 32 * wq + lane;
+                if (valid < kTile && r >= valid) {
+                    const uint32_t R = static_cast<uint32_t>(p.ring);
+#pragma unroll 1
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t ra = sm.slot(static_cast<int>((kF8Units * it + j) % R)) + r * 128u;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) ptx::st_shared_v4(ra + 16u * c, 0u, 0u, 0u, 0u);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t pk[NG][2];
+#pragma unroll
+                    for (int gi = 0; gi < NG; ++gi) {
+                        const float p0 = ptx::ex2_approx(d[hf][gi][0]);  // masked entries: 2^-inf = 0
+                        const float p1 = ptx::ex2_approx(d[hf][gi][1]);
+                        const float p2 = ptx::ex2_approx(d[hf][gi][2]);
+                        const float p3 = ptx::ex2_approx(d[hf][gi][3]);
+                        l[gi][0] += p0 + p2;
+                        l[gi][1] += p1 + p3;
                         pk[gi][0] = ptx::pack_bf16x2(p0, p1);  // token row r8
                         pk[gi][1] = ptx::pack_bf16x2(p2, p3);  // token row r8 + 8
                     }
-                }
-                // P^T rows n, K positions = tokens of the tile (natural order)
-                const int kb = 32 * wq + 16 * hf + 8 * st_blk;  // first token of this lane's matrix
-                const uint32_t kbase = pbuf + (kb >> 6) * C::QCHUNK;
-                const uint32_t kchunk = static_cast<uint32_t>((kb & 63) >> 3);
+                    // P^T rows n, K positions = tokens of the tile (natural order)
+                    const int kb = 32 * wq + 16 * hf + 8 * st_blk;  // first token of this lane's matrix
+                    const uint32_t kbase = pbuf + (kb >> 6) * C::QCHUNK;
+                    const uint32_t kchunk = static_cast<uint32_t>((kb & 63) >> 3);
 #pragma unroll
-                for (int gp = 0; gp < NG / 2; ++gp) {
-                    const int n = 8 * (2 * gp + st_go) + st_row;
-                    const uint32_t addr = kbase + n * 128u + ((kchunk ^ static_cast<uint32_t>(n & 7)) << 4);
-                    ptx::stsm_x4_trans(addr, pk[2 * gp][0], pk[2 * gp][1], pk[2 * gp + 1][0], pk[2 * gp + 1][1]);
+                    for (int gp = 0; gp < NG / 2; ++gp) {
+                        const int n = 8 * (2 * gp + st_go) + st_row;
+                        const uint32_t addr = kbase + n * 128u + ((kchunk ^ static_cast<uint32_t>(n & 7)) << 4);
+                        ptx::stsm_x4_trans(addr, pk[2 * gp][0], pk[2 * gp][1], pk[2 * gp + 1][0], pk[2 * gp + 1][1]);
+                    }
                 }
             }
             ptx::fence_proxy_async_smem();
@@ -1267,9 +1451,9 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     sm.ring = base;
-    sm.slot_bytes = C::SLOT_BYTES;
-    uint32_t off = p.ring * C::SLOT_BYTES;
-    if constexpr (F8) off += kF8Stage * kF8StageBytes;  // FP8: the staging ring, then the token scales
+    sm.slot_bytes = F8 ? kF8UnitBytes : C::SLOT_BYTES;
+    uint32_t off = p.ring * (F8 ? kF8UnitBytes : C::SLOT_BYTES);
+    if constexpr (F8) off += kQsBytes;  // FP8: the ring of units, the q terms, then the token scales
     sm.f8 = base + off;
     if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
@@ -1283,19 +1467,18 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.tmem_holder = reinterpret_cast<uint32_t *>(sm.shift + N);
     sm.abort_flag = reinterpret_cast<volatile int *>(sm.tmem_holder + 1);
     sm.scratch = ptx::smem_addr(sm.tmem_holder + 4);
-    sm.tscale = reinterpret_cast<float *>(misc + misc_bytes<N>());  // FP8 only: kScBytes past the misc region
+    sm.tscale = reinterpret_cast<float *>(misc + misc_bytes<N>());  // FP8 only: q scales, past the misc region
 
     const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ring; ++s) {
-            ptx::mbar_init(sm.bar(kBarFull + s), F8 ? 4 : 1);  // FP8: the four converter warps
-            ptx::mbar_init(sm.bar(kBarEmpty + s), C::EMPTY_ARRIVALS);
+            ptx::mbar_init(sm.bar(kBarFull + s), 1);
+            // FP8: a unit's slot is free after the score and the output MMA
+            // (the rope unit: two commits of the score MMA)
+            ptx::mbar_init(sm.bar(kBarEmpty + s), F8 ? 2 : C::EMPTY_ARRIVALS);
         }
         if constexpr (F8) {
-            for (int s = 0; s < kF8Stage; ++s) {
-                ptx::mbar_init(sm.bar(kBarRawFull + s), 1);
-                ptx::mbar_init(sm.bar(kBarRawEmpty + s), 4);
-            }
+            ptx::mbar_init(sm.bar(kBarQsFull), 4);  // one arrival per softmax warp
         } else {
             // (unused by the bf16 instances; kept so their set-up is unchanged)
             for (int i = 0; i < 4; ++i) {
@@ -1383,11 +1566,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
     if (decode_setup<N, SQ, F8>(p, &kv_map, &q_map, &sc_map, smem_raw, sm, w, tmem)) {
         const int warp = threadIdx.x >> 5;
         const int g = blockIdx.x % p.G;
-        if (warp == 0) producer_warp<N, SQ, F8>(p, w, g, sm, &kv_map, &q_map, &sc_map);
-        else if (warp == 1) score_mma_warp<N, SQ>(p, w, sm, tmem);
-        else if (warp < 6) softmax_warps<N, SQ, F8>(p, w, g, sm, tmem);
-        else if (warp < 10) transposer_warps<N, SQ, F8>(p, w, sm, tmem);
-        else output_mma_warp<N, SQ>(p, w, sm, tmem);
+        if (warp == 0) {
+            producer_warp<N, SQ, F8>(p, w, g, sm, &kv_map, &q_map, &sc_map);
+        } else if (warp == 1) {
+            if constexpr (F8) score_mma_warp_f8<N, SQ>(p, w, sm, tmem);
+            else score_mma_warp<N, SQ>(p, w, sm, tmem);
+        } else if (warp < 6) {
+            softmax_warps<N, SQ, F8>(p, w, g, sm, tmem);
+        } else if (warp < 10) {
+            transposer_warps<N, SQ, F8>(p, w, sm, tmem);
+        } else {
+            if constexpr (F8) output_mma_warp_f8<N, SQ>(p, w, sm, tmem);
+            else output_mma_warp<N, SQ>(p, w, sm, tmem);
+        }
     }
     decode_teardown<N, SQ>(tmem);
 }
@@ -1669,10 +1860,16 @@ int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
     const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024 +
-                                       (F8 ? kF8Stage * kF8StageBytes + kRawScBytes + kScBytes : 0));
-    int R = (smem_optin - fixed) / static_cast<int>(C::SLOT_BYTES);
+                                       (F8 ? kQsBytes + kRawScBytes + kScBytes : 0));
+    const uint32_t slot = F8 ? kF8UnitBytes : C::SLOT_BYTES;
+    int R = (smem_optin - fixed) / static_cast<int>(slot);
     if (R > kMaxRing) R = kMaxRing;
-    *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * C::SLOT_BYTES;
+    // FP8: the token scales of tile T + 4 replace tile T's once the slot of
+    // unit 5 (T + 4) - R is free; for 7 <= R <= 10 that unit is a latent unit
+    // of tile T + 2 or T + 1, freed only after the softmax of tile T has read
+    // its scales.
+    if (F8 && R > 10) R = 10;
+    *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * slot;
     return R;
 }
 
@@ -1703,7 +1900,7 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
     }
     size_t smem = 0;
     const int R = ring_for<N, SQ, F8>(info.smem_optin, &smem);
-    if (R * Cfg<N, SQ>::CPS < kMinRingChunks) {
+    if (R * Cfg<N, SQ>::CPS < kMinRingChunks || (F8 && R < 7)) {
         snprintf(g_last_error, sizeof g_last_error, "not enough shared memory for a %d-chunk ring", kMinRingChunks);
         return MLA_ERR_CUDA;
     }
