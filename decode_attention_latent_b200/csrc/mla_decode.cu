@@ -449,6 +449,9 @@ struct Cfg {
     static constexpr uint32_t QBYTES = kChunks * QCHUNK;   // N x 576 bf16
     static constexpr uint32_t PBYTES = 2 * 2 * QCHUNK;     // 2 P^T buffers of N x 128 bf16
     static constexpr uint32_t S_COL = 4 * N;
+    // FP8 instance: each MMA has 2N columns, n and N + n holding the hi and
+    // lo terms of column n; O^T blocks are 2N wide, S^T from column 8N.
+    static constexpr uint32_t S_COL8 = 8 * N;
     static constexpr uint32_t VT_COL = (S_COL + NS * N + 63) / 64 * 64;
     static constexpr int NVT = (512 - static_cast<int>(VT_COL)) / 64;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -491,7 +494,7 @@ struct Smem {
 // piece for the combine kernel.  O^T must be complete (and fenced) when this
 // is called.  `l` holds the calling thread's partial sums in the fragment
 // layout of softmax_warps.
-template <int N, int SQ>
+template <int N, int SQ, bool F8 = false>
 __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t tmem, int b, int split, int g,
                                const float (&l)[N / 8][2])
 {
@@ -559,9 +562,23 @@ __device__ void range_epilogue(const DecodeParams &p, const Smem &sm, uint32_t t
 #pragma unroll
         for (int c0 = 0; c0 < N; c0 += CW) {
             float v[CW / 16][16];
+            if constexpr (F8) {  // block j is 2N wide: add its hi and lo halves
+                float u[CW / 16][16];
 #pragma unroll
-            for (int k = 0; k < CW / 16; ++k) ptx::tmem_ld16(tmem + lane_base + j * N + c0 + 16 * k, v[k]);
-            ptx::tmem_wait_ld();
+                for (int k = 0; k < CW / 16; ++k) {
+                    ptx::tmem_ld16(tmem + lane_base + j * 2 * N + c0 + 16 * k, v[k]);
+                    ptx::tmem_ld16(tmem + lane_base + j * 2 * N + N + c0 + 16 * k, u[k]);
+                }
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < CW / 16; ++k)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[k][e] += u[k][e];
+            } else {
+#pragma unroll
+                for (int k = 0; k < CW / 16; ++k) ptx::tmem_ld16(tmem + lane_base + j * N + c0 + 16 * k, v[k]);
+                ptx::tmem_wait_ld();
+            }
             if (final_out) {
 #pragma unroll
                 for (int e = 0; e < CW; ++e) {
@@ -811,14 +828,16 @@ __device__ void output_mma_warp(const DecodeParams &p, const Range &w, const Sme
 
 // -- FP8 cache: the two MMA warps on the e4m3 codes ------------------------
 // Score MMA: S^T(t) = sum over the tile's five units of K_unit q_unit^T, with
-// q as its two e4m3 terms (hi, lo), K = 32 codes per instruction.  Latent
+// q as its two e4m3 terms stacked as 2N rows (hi rows 0..N-1, lo rows N..2N-1,
+// so S^T has 2N columns whose halves the softmax adds), K = 32 codes per
+// instruction.  Latent
 // units stay in the ring for the output MMA; the rope unit is free after the
 // score MMA (both of its slot's arrivals come from here).
 template <int N, int SQ>
 __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
-    constexpr uint32_t idS = ptx::idesc_e4m3_f32(128, N, false, false);  // codes K-major, q terms K-major
+    constexpr uint32_t idS = ptx::idesc_e4m3_f32(128, 2 * N, false, false);  // codes K-major, q terms K-major
     const uint32_t R = static_cast<uint32_t>(p.ring);
     const uint32_t qs = sm.f8 - kQsBytes;
     uint32_t cc = 0, it = 0;
@@ -837,7 +856,7 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
             const uint32_t sb = it % C::NS, su = it / C::NS;
             if (su >= 1 && !(ok = warp_wait(sm.bar(kBarSEmpty + sb), (su & 1) ^ 1, sm.abort_flag, p.err))) break;
             ptx::tc_fence_after();
-            const uint32_t d = tmem + C::S_COL + sb * N;
+            const uint32_t d = tmem + C::S_COL8 + sb * 2 * N;
 #pragma unroll 1
             for (int k = 0; k < kF8Units; ++k) {
                 const uint32_t u = cc + k;
@@ -849,11 +868,8 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
                 const int steps = (k == kF8Units - 1) ? 2 : 4;  // the rope unit: 64 columns
 #pragma unroll 1
                 for (int kk = 0; kk < steps; ++kk)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        ptx::mma_e4m3_ss_elect(d, ptx::desc_sw128(a0 + 32u * kk, 16, 1024),
-                                               ptx::desc_sw128(q0 + h * 2048u + 32u * kk, 16, 1024), idS,
-                                               (k | kk | h) != 0);
+                    ptx::mma_e4m3_ss_elect(d, ptx::desc_sw128(a0 + 32u * kk, 16, 1024),
+                                           ptx::desc_sw128(q0 + 32u * kk, 16, 1024), idS, (k | kk) != 0);
                 ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
                 if (k == kF8Units - 1) ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
             }
@@ -869,14 +885,15 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
 }
 
 // Output MMA: O^T block j += V^T_j P~^T, V^T_j = latent unit j of the tile read
-// MN-major straight from its ring slot, P~ the weights as two e4m3 terms (hi,
-// lo: N rows x 128 tokens each, K-major), 32 tokens per instruction.  Each
-// unit's slot is free once its MMAs are complete.
+// MN-major straight from its ring slot, P~ the weights as two e4m3 terms
+// stacked as 2N rows of 128 tokens (K-major), 32 tokens per instruction; the
+// epilogue adds the block's two column halves.  Each unit's slot is free once
+// its MMAs are complete.
 template <int N, int SQ>
 __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
-    constexpr uint32_t idO = ptx::idesc_e4m3_f32(128, N, true, false);  // V^T MN-major, P~^T K-major
+    constexpr uint32_t idO = ptx::idesc_e4m3_f32(128, 2 * N, true, false);  // V^T MN-major, P~^T K-major
     const uint32_t R = static_cast<uint32_t>(p.ring);
     uint32_t it = 0, cc = 0;
     bool ok = true;
@@ -900,11 +917,8 @@ __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const 
                 const uint32_t a0 = sm.slot(slot);
 #pragma unroll 1
                 for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        ptx::mma_e4m3_ss_elect(tmem + j * N, ptx::desc_sw128(a0 + 4096u * kk, 8192, 1024),
-                                               ptx::desc_sw128(pa + h * 2048u + 32u * kk, 16, 1024), idO,
-                                               (t != tb) || kk != 0 || h != 0);
+                    ptx::mma_e4m3_ss_elect(tmem + j * 2 * N, ptx::desc_sw128(a0 + 4096u * kk, 8192, 1024),
+                                           ptx::desc_sw128(pa + 32u * kk, 16, 1024), idO, (t != tb) || kk != 0);
                 ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
             }
             if (!ok) break;
@@ -1192,11 +1206,27 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             wait_ok = wait_bounded(sm.bar(kBarSFull + sb), su & 1, sm.abort_flag, p.err) && wait_ok;
             ptx::tc_fence_after();
             uint32_t raw[2][4 * NG];
+            if constexpr (F8) {  // the hi and lo halves of S^T
+                uint32_t lo[2][4 * NG];
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-                ptx::tmem_ld_16x256b(tmem + (static_cast<uint32_t>(32 * wq + 16 * hf) << 16) + C::S_COL + sb * N,
-                                     raw[hf]);
-            ptx::tmem_wait_ld();
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t ta = tmem + (static_cast<uint32_t>(32 * wq + 16 * hf) << 16) + C::S_COL8 + sb * 2 * N;
+                    ptx::tmem_ld_16x256b(ta, raw[hf]);
+                    ptx::tmem_ld_16x256b(ta + N, lo[hf]);
+                }
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int i = 0; i < 4 * NG; ++i)
+                        raw[hf][i] = __float_as_uint(__uint_as_float(raw[hf][i]) + __uint_as_float(lo[hf][i]));
+            } else {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                    ptx::tmem_ld_16x256b(tmem + (static_cast<uint32_t>(32 * wq + 16 * hf) << 16) + C::S_COL + sb * N,
+                                         raw[hf]);
+                ptx::tmem_wait_ld();
+            }
             // S^T(it) is in registers: its TMEM buffer may be overwritten
             ptx::tc_fence_before();
             __syncwarp();
@@ -1323,7 +1353,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                             a[4 * e4 + 3] = ptx::ex2_approx(-v4.w);
                         }
 #pragma unroll 1
-                        for (int j = 0; j < 4; ++j) {
+                        for (int j = 0; j < (F8 ? 8 : 4); ++j) {  // FP8: both halves of the 4 blocks
                             float x[16];
                             const uint32_t ta = tmem + lane_base + j * N + ch * 16;
                             ptx::tmem_ld16(ta, x);
@@ -1431,7 +1461,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         __syncwarp();
         if (!(ok = ptx::named_bar_and(1, 128, wait_ok))) break;
         ptx::tc_fence_after();
-        range_epilogue<N, SQ>(p, sm, tmem, b, split, g, l);
+        range_epilogue<N, SQ, F8>(p, sm, tmem, b, split, g, l);
     }
 }
 
