@@ -98,10 +98,14 @@ constexpr int kBarDrainO = kBarDrain + 1;
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
 constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
 constexpr uint32_t kF8UnitBytes = 16384;   // one ring slot: a unit's codes
-constexpr int kRawScBufs = 4;
+// Token scales of tile T are replaced by tile T + 8's once the slot of unit
+// 5 (T + 8) - R is free: for R <= 16 a unit of tile T + 5 or later, freed only
+// after the softmax of tile T has read them.
+constexpr int kRawScBufs = 8;
 constexpr uint32_t kRawScBytes = kRawScBufs * 512;
 // q split into two e4m3 terms per element (see softmax_warps), per unit a hi
-// and a lo tile of 16 rows x 128 B, 128-byte swizzled, K-major.
+// and a lo tile of 16 rows x 128 B, 128-byte swizzled, K-major.  The bf16 q
+// is loaded into the same bytes and split in place.
 constexpr uint32_t kQsUnitBytes = 4096;
 constexpr uint32_t kQsBytes = kF8Units * kQsUnitBytes;
 // FP8 weights: the reference max sits kLift8 below the largest log2 weight
@@ -117,7 +121,8 @@ constexpr float kTau8 = 8.f;
 constexpr int kBarF8Full = kBarDrainO + 1;
 constexpr int kBarQsFull = kBarF8Full;
 constexpr int kScBufs = 4;
-constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // FP8: per-row q scales (first 16 words)
+constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // (unused; kept for the layout of the bf16 instances)
+constexpr uint32_t kQScaleBytes = 128;              // FP8: the per-row q scales
 constexpr int kBarF8Reserved = kBarF8Full + 8 + 2 * kScBufs;
 constexpr int kNumBars = kBarF8Reserved;
 // The reduction buffers after the barriers are read as float4: keep them
@@ -839,7 +844,7 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
     using C = Cfg<N, SQ>;
     constexpr uint32_t idS = ptx::idesc_e4m3_f32(128, 2 * N, false, false);  // codes K-major, q terms K-major
     const uint32_t R = static_cast<uint32_t>(p.ring);
-    const uint32_t qs = sm.f8 - kQsBytes;
+    const uint32_t qs = sm.q;
     uint32_t cc = 0, it = 0;
     int qi = 0;
     bool ok = true;
@@ -1105,16 +1110,19 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     // columns are multiplied back by 2^-a_n (Smem::tscale[n]).  Thread: row
     // n = stid / 8 and the 16-column groups stid % 8 + 8 i, i < 5 (groups
     // 36-39 are the zero fill past column 575 that the rope unit's upper
-    // half meets).
+    // half meets).  The bf16 q lies in the same bytes (nine 2 KB chunks of
+    // 64 columns); unit i's hi and lo tiles cover chunks 2i and 2i + 1, and
+    // row n of them only row n of those chunks, which the row's eight
+    // threads (one warp) read before any of them writes.
     uint32_t qsplits = 0;
     auto split_q = [&]() -> bool {
         const bool okq = wait_bounded(sm.bar(kBarQFull), qsplits & 1, sm.abort_flag, p.err);
         ++qsplits;
         const int n = stid >> 3, part = stid & 7;
-        const uint32_t qs = sm.f8 - kQsBytes;
+        const uint32_t qs = sm.q;
         auto load16 = [&](int gq, float (&v)[16]) {
             const int c = gq >> 2, u0 = (gq & 3) * 2;
-            const uint32_t rowa = sm.q + c * C::QCHUNK + n * 128u;
+            const uint32_t rowa = qs + c * C::QCHUNK + n * 128u;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const uint4 x = ptx::ld_shared_v4(rowa + ((static_cast<uint32_t>(u0 + hh) ^ (n & 7)) << 4));
@@ -1152,6 +1160,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 #pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] = 0.f;
             }
+            __syncwarp();  // the row's bf16 values of unit i are in registers
             uint32_t hw[4], lw[4];
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
@@ -1167,8 +1176,8 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                 hw[e4] = hb[0] | (hb[1] << 16);
                 lw[e4] = lb[0] | (lb[1] << 16);
             }
-            const uint32_t at = qs + (gq >> 3) * kQsUnitBytes + n * 128u +
-                                ((static_cast<uint32_t>(gq & 7) ^ static_cast<uint32_t>(n & 7)) << 4);
+            const uint32_t at = qs + i * kQsUnitBytes + n * 128u +
+                                ((static_cast<uint32_t>(part) ^ static_cast<uint32_t>(n & 7)) << 4);
             ptx::st_shared_v4(at, hw[0], hw[1], hw[2], hw[3]);
             ptx::st_shared_v4(at + 2048u, lw[0], lw[1], lw[2], lw[3]);
         }
@@ -1483,12 +1492,12 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.ring = base;
     sm.slot_bytes = F8 ? kF8UnitBytes : C::SLOT_BYTES;
     uint32_t off = p.ring * (F8 ? kF8UnitBytes : C::SLOT_BYTES);
-    if constexpr (F8) off += kQsBytes;  // FP8: the ring of units, the q terms, then the token scales
-    sm.f8 = base + off;
+    sm.f8 = base + off;  // FP8: the ring of units, the token scales, then q (split in place) and P~^T
     if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
-    sm.p = sm.q + C::QBYTES;
-    uint8_t *misc = gbase + off + C::QBYTES + C::PBYTES;
+    constexpr uint32_t qreg = F8 ? kQsBytes : C::QBYTES;
+    sm.p = sm.q + qreg;
+    uint8_t *misc = gbase + off + qreg + C::PBYTES;
     sm.bars = ptx::smem_addr(misc);
     sm.red = reinterpret_cast<float *>(misc + kMiscRedOffset);
     sm.lred = sm.red + 4 * N;
@@ -1889,16 +1898,11 @@ template <int N, int SQ, bool F8>
 int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
-    const int fixed = static_cast<int>(C::QBYTES + C::PBYTES + misc_bytes<N>() + 1024 +
-                                       (F8 ? kQsBytes + kRawScBytes + kScBytes : 0));
+    const int fixed = static_cast<int>((F8 ? kQsBytes : C::QBYTES) + C::PBYTES + misc_bytes<N>() + 1024 +
+                                       (F8 ? kRawScBytes + kQScaleBytes : 0));
     const uint32_t slot = F8 ? kF8UnitBytes : C::SLOT_BYTES;
     int R = (smem_optin - fixed) / static_cast<int>(slot);
     if (R > kMaxRing) R = kMaxRing;
-    // FP8: the token scales of tile T + 4 replace tile T's once the slot of
-    // unit 5 (T + 4) - R is free; for 7 <= R <= 10 that unit is a latent unit
-    // of tile T + 2 or T + 1, freed only after the softmax of tile T has read
-    // its scales.
-    if (F8 && R > 10) R = 10;
     *smem_bytes = static_cast<size_t>(fixed) + static_cast<size_t>(R) * slot;
     return R;
 }
@@ -1930,7 +1934,7 @@ mla_status_t launch_decode(const CUtensorMap &kv_map, const CUtensorMap &q_map, 
     }
     size_t smem = 0;
     const int R = ring_for<N, SQ, F8>(info.smem_optin, &smem);
-    if (R * Cfg<N, SQ>::CPS < kMinRingChunks || (F8 && R < 7)) {
+    if (R * Cfg<N, SQ>::CPS < kMinRingChunks || (F8 && R < kF8Units)) {
         snprintf(g_last_error, sizeof g_last_error, "not enough shared memory for a %d-chunk ring", kMinRingChunks);
         return MLA_ERR_CUDA;
     }
