@@ -249,7 +249,8 @@ def decode_fp8(q: torch.Tensor, kv_codes: torch.Tensor, kv_scale: torch.Tensor, 
                combine: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
     """MLA decode over an FP8 cache (``mla_decode_fp8``): ``kv_codes`` uint8
     [num_blocks, 64, 576] e4m3 codes, ``kv_scale`` fp32 [num_blocks, 64], one
-    scale per cached token.  s_q = 1, H = 16."""
+    scale per cached token.  16 or 32 query columns: H = 16 with s_q = 1 or
+    2, or H = 32 with s_q = 1."""
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("q must be a CUDA tensor")

@@ -103,11 +103,10 @@ constexpr uint32_t kF8UnitBytes = 16384;   // one ring slot: a unit's codes
 // after the softmax of tile T has read them.
 constexpr int kRawScBufs = 8;
 constexpr uint32_t kRawScBytes = kRawScBufs * 512;
-// q split into two e4m3 terms per element (see softmax_warps), per unit a hi
-// and a lo tile of 16 rows x 128 B, 128-byte swizzled, K-major.  The bf16 q
-// is loaded into the same bytes and split in place.
-constexpr uint32_t kQsUnitBytes = 4096;
-constexpr uint32_t kQsBytes = kF8Units * kQsUnitBytes;
+// q split into two e4m3 terms per element (see softmax_warps): per unit a hi
+// and a lo tile of N rows x 128 B each, stacked, 128-byte swizzled, K-major
+// (Cfg::QS8_UNIT, Cfg::QS8).  The bf16 q is loaded into the same bytes and
+// split in place.
 // FP8 weights: the reference max sits kLift8 below the largest log2 weight
 // seen when it last moved, so weights reach 2^kLift8 and stay above e4m3's
 // subnormal range (2^-6) down to 2^-13 of the largest; it moves again when a
@@ -457,6 +456,8 @@ struct Cfg {
     // FP8 instance: each MMA has 2N columns, n and N + n holding the hi and
     // lo terms of column n; O^T blocks are 2N wide, S^T from column 8N.
     static constexpr uint32_t S_COL8 = 8 * N;
+    static constexpr uint32_t QS8_UNIT = 2 * N * 128u;        // FP8: one unit of q's stacked e4m3 terms
+    static constexpr uint32_t QS8 = kF8Units * QS8_UNIT;       // holds the bf16 q too (9 x 128 N bytes)
     static constexpr uint32_t VT_COL = (S_COL + NS * N + 63) / 64 * 64;
     static constexpr int NVT = (512 - static_cast<int>(VT_COL)) / 64;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -869,7 +870,7 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
                 if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
                 ptx::tc_fence_after();
                 const uint32_t a0 = sm.slot(slot);
-                const uint32_t q0 = qs + k * kQsUnitBytes;
+                const uint32_t q0 = qs + k * C::QS8_UNIT;
                 const int steps = (k == kF8Units - 1) ? 2 : 4;  // the rope unit: 64 columns
 #pragma unroll 1
                 for (int kk = 0; kk < steps; ++kk)
@@ -1107,18 +1108,21 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
     // has at most four significant bits, so hi + lo = x exactly unless lo
     // falls below the e4m3 normal range (|x| < 2^-2, i.e. 2^-10 of the row's
     // largest value), where lo keeps its bits down to 2^-9.  The score
-    // columns are multiplied back by 2^-a_n (Smem::tscale[n]).  Thread: row
-    // n = stid / 8 and the 16-column groups stid % 8 + 8 i, i < 5 (groups
-    // 36-39 are the zero fill past column 575 that the rope unit's upper
-    // half meets).  The bf16 q lies in the same bytes (nine 2 KB chunks of
-    // 64 columns); unit i's hi and lo tiles cover chunks 2i and 2i + 1, and
-    // row n of them only row n of those chunks, which the row's eight
-    // threads (one warp) read before any of them writes.
+    // columns are multiplied back by 2^-a_n (Smem::tscale[n]).  Row n has
+    // 128 / N threads (one warp holds whole rows); of each unit's eight
+    // 16-column groups a thread takes 8 N / 128 (groups 36-39, past column
+    // 575, are the zero fill the rope unit's upper half meets).  The bf16 q
+    // lies in the same bytes (nine chunks of 64 columns, N rows x 128 B
+    // each); unit u's hi and lo tiles cover chunks 2u and 2u + 1, and row n of
+    // them only row n of those chunks, which the row's threads read before
+    // any of them writes.
+    constexpr int TPR = 128 / N;  // threads per q row
+    constexpr int GPU = 8 / TPR;  // 16-column groups per unit and thread
     uint32_t qsplits = 0;
     auto split_q = [&]() -> bool {
         const bool okq = wait_bounded(sm.bar(kBarQFull), qsplits & 1, sm.abort_flag, p.err);
         ++qsplits;
-        const int n = stid >> 3, part = stid & 7;
+        const int n = stid / TPR, part = stid % TPR;
         const uint32_t qs = sm.q;
         auto load16 = [&](int gq, float (&v)[16]) {
             const int c = gq >> 2, u0 = (gq & 3) * 2;
@@ -1136,50 +1140,58 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
         };
         float mx = 0.f;
 #pragma unroll 1
-        for (int i = 0; i < 5; ++i) {
-            const int gq = part + 8 * i;
-            if (gq >= 36) continue;
-            float v[16];
-            load16(gq, v);
+        for (int u = 0; u < kF8Units; ++u)
 #pragma unroll
-            for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            for (int e = 0; e < GPU; ++e) {
+                const int gq = 8 * u + part + TPR * e;
+                if (gq >= 36) continue;
+                float v[16];
+                load16(gq, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
+            }
+#pragma unroll
+        for (int o = 1; o < TPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         int ex = 0;
         frexpf(mx, &ex);  // mx < 2^ex
         const float up = ldexpf(1.f, 8 - ex);
 #pragma unroll 1
-        for (int i = 0; i < 5; ++i) {
-            const int gq = part + 8 * i;
-            float v[16];
-            if (gq < 36) {
-                load16(gq, v);
-            } else {
+        for (int u = 0; u < kF8Units; ++u) {
+            float v[GPU][16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            }
-            __syncwarp();  // the row's bf16 values of unit i are in registers
-            uint32_t hw[4], lw[4];
+            for (int e = 0; e < GPU; ++e) {
+                const int gq = 8 * u + part + TPR * e;
+                if (gq < 36) {
+                    load16(gq, v[e]);
+                } else {
 #pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-                uint32_t hb[2], lb[2];
-#pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const float x0 = v[4 * e4 + 2 * e2] * up, x1 = v[4 * e4 + 2 * e2 + 1] * up;
-                    hb[e2] = ptx::f32x2_to_e4m3x2(x0, x1);
-                    float h0, h1;
-                    ptx::e4m3x2_to_f32x2(hb[e2], h0, h1);
-                    lb[e2] = ptx::f32x2_to_e4m3x2(x0 - h0, x1 - h1);
+                    for (int i = 0; i < 16; ++i) v[e][i] = 0.f;
                 }
-                hw[e4] = hb[0] | (hb[1] << 16);
-                lw[e4] = lb[0] | (lb[1] << 16);
             }
-            const uint32_t at = qs + i * kQsUnitBytes + n * 128u +
-                                ((static_cast<uint32_t>(part) ^ static_cast<uint32_t>(n & 7)) << 4);
-            ptx::st_shared_v4(at, hw[0], hw[1], hw[2], hw[3]);
-            ptx::st_shared_v4(at + 2048u, lw[0], lw[1], lw[2], lw[3]);
+            __syncwarp();  // the row's bf16 values of unit u are in registers
+#pragma unroll
+            for (int e = 0; e < GPU; ++e) {
+                const int gq = 8 * u + part + TPR * e;
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    uint32_t hb[2], lb[2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const float x0 = v[e][4 * e4 + 2 * e2] * up, x1 = v[e][4 * e4 + 2 * e2 + 1] * up;
+                        hb[e2] = ptx::f32x2_to_e4m3x2(x0, x1);
+                        float h0, h1;
+                        ptx::e4m3x2_to_f32x2(hb[e2], h0, h1);
+                        lb[e2] = ptx::f32x2_to_e4m3x2(x0 - h0, x1 - h1);
+                    }
+                    hw[e4] = hb[0] | (hb[1] << 16);
+                    lw[e4] = lb[0] | (lb[1] << 16);
+                }
+                const uint32_t at = qs + u * C::QS8_UNIT + n * 128u +
+                                    ((static_cast<uint32_t>(gq & 7) ^ static_cast<uint32_t>(n & 7)) << 4);
+                ptx::st_shared_v4(at, hw[0], hw[1], hw[2], hw[3]);
+                ptx::st_shared_v4(at + N * 128u, lw[0], lw[1], lw[2], lw[3]);
+            }
         }
         if (part == 0) sm.tscale[n] = ldexpf(1.f, ex - 8);
         ptx::fence_proxy_async_smem();
@@ -1245,7 +1257,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
             const bool first = (t == tb);
             const int tok0 = t * kTile + 32 * wq + r8;
             // FP8 cache: the scales of this thread's four token rows (0 for rows
-            // past the visible tokens), from the buffer that landed with the
+            // past the sequence's end), from the buffer that landed with the
             // tile's first unit (which the score MMA waited for).  A token's
             // weight in O is 2^(x - mu) tsc with x its log2-domain score;
             // the reference max mu follows x + log2|tsc|, so that weight is
@@ -1260,7 +1272,7 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const int row = 32 * wq + r8 + 16 * hf + 8 * jj;
-                        const float x = (tok0 + 16 * hf + 8 * jj < nvis0) ? ptx::ld_shared_f32(sbuf + 4u * row) : 0.f;
+                        const float x = (tok0 + 16 * hf + 8 * jj < L) ? ptx::ld_shared_f32(sbuf + 4u * row) : 0.f;
                         tsc[hf][jj] = x;
                         lgt[hf][jj] = x != 0.f ? __log2f(fabsf(x)) : 0.f;
                         sgt[hf][jj] = x > 0.f ? 1.f : (x < 0.f ? -1.f : 0.f);
@@ -1386,8 +1398,8 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                 // FP8: l takes 2^(x - mu); O takes w = 2^(x - mu) tsc as two
                 // e4m3 terms, hi = e4m3(w) and lo = e4m3(w - hi) (8 significant
                 // bits together, like bf16), written as P~^T (row n, token k at
-                // n * 128 + ((k / 16) ^ (n % 8)) * 16 + k % 16; hi at pbuf, lo
-                // 2 KB after it)
+                // n * 128 + ((k / 16) ^ (n % 8)) * 16 + k % 16; hi rows n, lo rows
+                // N + n)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -1413,8 +1425,8 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                                                 static_cast<uint32_t>(k & 15);
                             ptx::st_shared_u8(a0, hb & 0xFFu);
                             ptx::st_shared_u8(a1, hb >> 8);
-                            ptx::st_shared_u8(a0 + 2048u, lb & 0xFFu);
-                            ptx::st_shared_u8(a1 + 2048u, lb >> 8);
+                            ptx::st_shared_u8(a0 + N * 128u, lb & 0xFFu);
+                            ptx::st_shared_u8(a1 + N * 128u, lb >> 8);
                         }
                 // Rows past the sequence's end in its last tile hold whatever the
                 // cache (or an earlier unit) left there, NaN codes included; their
@@ -1495,7 +1507,7 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.f8 = base + off;  // FP8: the ring of units, the token scales, then q (split in place) and P~^T
     if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
-    constexpr uint32_t qreg = F8 ? kQsBytes : C::QBYTES;
+    constexpr uint32_t qreg = F8 ? C::QS8 : C::QBYTES;
     sm.p = sm.q + qreg;
     uint8_t *misc = gbase + off + qreg + C::PBYTES;
     sm.bars = ptx::smem_addr(misc);
@@ -1875,7 +1887,7 @@ bool tensor_map(CUtensorMap *out, const char *what, CUtensorMapDataType dtype, i
 struct DeviceInfo {
     int smem_optin = 0;
     int major = 0;
-    bool attr_set[8] = {false, false, false, false, false, false, false, false};
+    bool attr_set[10] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -1884,7 +1896,7 @@ DeviceInfo g_dev[64];
 template <int N, int SQ, bool F8>
 int kernel_index()
 {
-    if (F8) return 7;
+    if (F8) return N == 16 ? 7 : (SQ == 1 ? 8 : 9);
     if (N == 16 && SQ == 1) return 0;
     if (N == 32 && SQ == 1) return 1;
     if (N == 32 && SQ == 2) return 2;
@@ -1898,7 +1910,7 @@ template <int N, int SQ, bool F8>
 int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
-    const int fixed = static_cast<int>((F8 ? kQsBytes : C::QBYTES) + C::PBYTES + misc_bytes<N>() + 1024 +
+    const int fixed = static_cast<int>((F8 ? C::QS8 : C::QBYTES) + C::PBYTES + misc_bytes<N>() + 1024 +
                                        (F8 ? kRawScBytes + kQScaleBytes : 0));
     const uint32_t slot = F8 ? kF8UnitBytes : C::SLOT_BYTES;
     int R = (smem_optin - fixed) / static_cast<int>(slot);
@@ -2065,7 +2077,8 @@ mla_status_t check_decode_args(const void *q, const void *kv, const void *kv_sca
         return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (!resolve(s_q, H, sh)) return MLA_ERR_UNSUPPORTED_SHAPE;
-    if (fp8 && (sh->N != 16 || s_q != 1)) return MLA_ERR_UNSUPPORTED_SHAPE;
+    // FP8 cache: 16 or 32 query columns (H = 16 with s_q = 1 or 2, H = 32 with s_q = 1)
+    if (fp8 && !(sh->G == 1 && (sh->N == 16 || (sh->N == 32 && s_q <= 2)))) return MLA_ERR_UNSUPPORTED_SHAPE;
     if (num_sms < sh->G || num_sms > kMaxSms) return MLA_ERR_UNSUPPORTED_SHAPE;
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(kv) & 15) ||
         (reinterpret_cast<uintptr_t>(kv_scale) & 15) || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
@@ -2170,8 +2183,12 @@ mla_status_t decode_fp8(const uint16_t *q, const uint8_t *kv_codes, const float 
     if (!q_tensor_map(&q_map, q, B, s_q, H, sh)) return MLA_ERR_CUDA;
     const DecodeParams prm = make_params(block_table, cache_seqlens, B, s_q, H, sh, num_blocks, max_blocks,
                                          softmax_scale, num_sms, sched_meta, num_splits, workspace, wl, out, lse);
-    const mla_status_t rc = launch_decode<16, 1, true>(kv_map, q_map, sc_map, prm, prm.num_tuples * sh.G,
-                                                       static_cast<cudaStream_t>(stream));
+    const int grid = prm.num_tuples * sh.G;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    mla_status_t rc;
+    if (sh.N == 16) rc = launch_decode<16, 1, true>(kv_map, q_map, sc_map, prm, grid, st);
+    else if (s_q == 1) rc = launch_decode<32, 1, true>(kv_map, q_map, sc_map, prm, grid, st);
+    else rc = launch_decode<32, 2, true>(kv_map, q_map, sc_map, prm, grid, st);
     if (rc != MLA_OK || !with_combine) return rc;
     return mla_decode_combine(num_splits, sched_meta, workspace, workspace_bytes, B, s_q, H, num_sms, out, lse,
                               stream);

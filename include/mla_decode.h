@@ -207,17 +207,20 @@ mla_status_t mla_decode_static_workspace(const uint16_t *q, const uint16_t *kv_c
  * per cached token: token j's row is e4m3(kv_codes[blk][j % 64][:]) *
  * kv_scale[blk][j % 64] (the juejin.cn "FlashMLA" post, section 5, says
  * FlashMLA runs in mixed precision such as FP8 and BF16; it fixes no format,
- * and this per-token-scale layout is the reading taken).  Each tile's codes
- * are widened in shared memory to bf16 (exactly: every e4m3 value is a bf16
- * value) for the tensor-core MMAs; each token's scale multiplies its scores
- * and its softmax weights in fp32, so the queries, the softmax and the
- * outputs are as in mla_decode.
+ * and this per-token-scale layout is the reading taken).  The tensor cores
+ * read the codes as they lie in the cache (tcgen05.mma kind::f8f6f4): each
+ * query row is written as two e4m3 terms whose sum is the bf16 row times a
+ * per-row power of two (exact but for values below 2^-10 of the row's
+ * largest), and each token's softmax weight, multiplied by its scale, as two
+ * e4m3 terms (8 significant bits, as a bf16 weight).  Scores, the softmax
+ * sums and the outputs are accumulated in fp32 as in mla_decode.  The two
+ * e4m3 NaN patterns (s.1111.111) are NaN.
  *   kv_codes   device uint8 [num_blocks, 64, 576] (e4m3 bit patterns, OCP E4M3
  *              as __nv_fp8_e4m3 holds them), 16-byte aligned.
  *   kv_scale   device fp32 [num_blocks, 64], 16-byte aligned.
  *   Every other argument as for mla_decode (same metadata, same workspace).
- * Supported shapes: s_q = 1 and H = 16 (16 query columns per CTA); others
- * return MLA_ERR_UNSUPPORTED_SHAPE.  mla_decode_attention_fp8 launches the
+ * Supported shapes: 16 or 32 query columns per CTA -- H = 16 with s_q = 1 or
+ * 2, H = 32 with s_q = 1; others return MLA_ERR_UNSUPPORTED_SHAPE.  mla_decode_attention_fp8 launches the
  * attention kernel alone, mla_decode_fp8 the attention and combine kernels. */
 mla_status_t mla_decode_attention_fp8(const uint16_t *q, const uint8_t *kv_codes, const float *kv_scale,
                                       const int32_t *block_table, const int32_t *cache_seqlens, int B, int s_q,

@@ -28,7 +28,7 @@ def orc():
 def run_fp8(inp, cache, dev, n_sms=None):
     q, bt, sl = inp.q.to(dev), inp.block_table.to(dev), inp.cache_seqlens.to(dev)
     n = mla.num_sms(dev) if n_sms is None else n_sms
-    sched, splits = mla.decode_metadata(sl, 1, inp.H, n)
+    sched, splits = mla.decode_metadata(sl, inp.s_q, inp.H, n)
     out, lse = mla.decode_fp8(q, cache.codes.to(dev), cache.scale.to(dev), bt, sl, inp.scale, sched_meta=sched,
                               num_splits=splits, num_sms_=n)
     err = mla.get_device_error(sched)
@@ -98,8 +98,39 @@ def test_fp8_paging_invariance(dev):
     assert np.array_equal(oa[0], ob[0]) and np.array_equal(oa[1], ob[1])
 
 
-def test_fp8_unsupported_shape_is_refused(dev):
-    inp = mi.small(B=1, s_q=1, H=32, seqlens=[100], seed=66)
+@pytest.mark.parametrize("H,s_q,seqlens,n_sms", [
+    (32, 1, [1, 200, 700], None), (32, 1, [64, 65, 127, 128, 129], 17),
+    (16, 2, [2, 200, 700], None), (16, 2, [64, 65, 127, 128, 129], 17), (16, 2, [64 * 40 + 3, 5000], 11),
+])
+def test_fp8_32_query_columns(dev, orc, H, s_q, seqlens, n_sms):
+    # 32 query columns: 32 heads, or 16 heads at two query positions (causal)
+    inp = mi.small(B=len(seqlens), s_q=s_q, H=H, seqlens=seqlens, seed=70)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=71)
+    g_out, g_lse, err = run_fp8(inp, cache, dev, n_sms)
+    assert err == 0
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"fp8 H={H} s_q={s_q} {seqlens}")
+
+
+def test_fp8_last_token_seen_by_the_second_query_position(dev, orc):
+    # s_q = 2: the last cached token is visible to query position 1 only; NaN
+    # codes and scales past the sequence end must still not reach the result
+    inp = mi.small(B=2, s_q=2, H=16, seqlens=[70, 129], seed=72)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=73)
+    for b, L in enumerate(inp.cache_seqlens.tolist()):
+        last = int(inp.block_table[b, (L - 1) // 64])
+        cache.codes[last, L % 64 or 64:, :] = 0x7F
+        cache.scale[last, L % 64 or 64:] = float("nan")
+        cache.scale[last, (L - 1) % 64] = 4.0  # the last token weighs in visibly for position 1
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err == 0 and np.all(np.isfinite(g_out)) and np.all(np.isfinite(g_lse))
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what="fp8 s_q=2 last token")
+
+
+@pytest.mark.parametrize("H,s_q", [(64, 1), (32, 2), (16, 4), (128, 1)])
+def test_fp8_unsupported_shape_is_refused(dev, H, s_q):
+    inp = mi.small(B=1, s_q=s_q, H=H, seqlens=[100], seed=66)
     cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=67)
     with pytest.raises(mla.MLAError):
         mla.decode_fp8(inp.q.to(dev), cache.codes.to(dev), cache.scale.to(dev), inp.block_table.to(dev),
