@@ -121,7 +121,8 @@ def test_decode_fp8_rejects_bad_arguments(lib):
                 P(GOOD), P(GOOD), P(0)]
     assert lib.mla_decode_fp8(*args(codes=0)) == 1
     assert lib.mla_decode_fp8(*args(scale=0)) == 1
-    assert lib.mla_decode_fp8(*args(H=32)) == 3      # 16 query columns only
+    assert lib.mla_decode_fp8(*args(H=64)) == 3      # 16 or 32 query columns only
+    assert lib.mla_decode_fp8(*args(H=16, s_q=4)) == 3
     assert lib.mla_decode_fp8(*args(s_q=2, H=8)) == 3
     assert lib.mla_decode_fp8(*args(codes=GOOD + 8)) == 2
     assert lib.mla_decode_fp8(*args(scale=GOOD + 4)) == 2
