@@ -664,7 +664,7 @@ def run_context_parallel_rank(args):
 
 def run_fp8(args):
     """The decode over an FP8 (e4m3, one fp32 scale per token) cache of the same
-    workload, one GPU: per call the metadata, attention and combine kernels
+    workload (16 or 32 query columns), one GPU: per call the metadata, attention and combine kernels
     (as the default line), the attention kernel alone and its roofline on
     576 + 4 bytes per cached token, and the error against the oracle's FP8
     definition."""
@@ -676,13 +676,13 @@ def run_fp8(args):
     torch.cuda.set_device(dev)
     lib = mla.load_library()
     w = selected_workload(args)
-    if w.s_q != 1 or w.H != 16:
-        raise SystemExit("the FP8 cache path takes s_q = 1, H = 16 workloads")
+    if w.s_q * w.H not in (16, 32) or w.s_q > 2:
+        raise SystemExit("the FP8 cache path takes 16 or 32 query columns (H = 16 with s_q <= 2, or H = 32)")
     inp = mi.make_inputs(w, seed=0)
     nb = inp.kv_cache.shape[0]
     inp.kv_cache = None  # the bf16 cache is not used here
     cache = mi.fp8_cache(nb, seed=1)
-    B, H = w.B, w.H
+    B, S, H = w.B, w.s_q, w.H
     n_sms = mla.num_sms(dev)
     fp8_bytes = nb * 64 * (576 + 4)
     n_copies = kv_copy_count(fp8_bytes, L2_BYTES)
@@ -691,21 +691,21 @@ def run_fp8(args):
     q, bt, sl = inp.q.to(dev), inp.block_table.to(dev), inp.cache_seqlens.to(dev)
     sched = torch.empty(mla.sched_meta_ints(n_sms), dtype=torch.int32, device=dev)
     splits = torch.empty(B + 1, dtype=torch.int32, device=dev)
-    ws_bytes = mla.workspace_size(B, 1, H, n_sms)
+    ws_bytes = mla.workspace_size(B, S, H, n_sms)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty(B, 1, H, mi.D_V, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(B, 1, H, dtype=torch.float32, device=dev)
+    out = torch.empty(B, S, H, mi.D_V, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, S, H, dtype=torch.float32, device=dev)
     sp = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     P = ctypes.c_void_p
 
     def meta():
-        assert lib.mla_decode_metadata(P(sl.data_ptr()), B, 1, H, n_sms, P(sched.data_ptr()),
+        assert lib.mla_decode_metadata(P(sl.data_ptr()), B, S, H, n_sms, P(sched.data_ptr()),
                                        P(splits.data_ptr()), sp) == 0
 
     def decode(k, fn):
         c, s_ = codes[k % n_copies], scales[k % n_copies]
         assert fn(P(q.data_ptr()), P(c.data_ptr()), P(s_.data_ptr()), P(bt.data_ptr()),
-                  P(sl.data_ptr()), B, 1, H, nb, bt.shape[1], ctypes.c_float(inp.scale),
+                  P(sl.data_ptr()), B, S, H, nb, bt.shape[1], ctypes.c_float(inp.scale),
                   n_sms, P(sched.data_ptr()), P(splits.data_ptr()), P(ws.data_ptr()),
                   ws_bytes, P(out.data_ptr()), P(lse.data_ptr()), sp) == 0
 
@@ -752,12 +752,13 @@ def run_fp8(args):
     line = {
         "metric": "MLA decode us/call over an FP8 (e4m3, per-token scale) cache", "value": call_us, "unit": "us/call",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
-        "dtype": "e4m3 cache, bf16 MMA", "data": "synthetic",
-        "config": {"workload": args.workload, "B": B, "H": H, "cache_copies": n_copies},
+        "dtype": "e4m3 cache and e4m3 MMA operands (q, weights as two e4m3 terms), fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "s_q": S, "H": H, "cache_copies": n_copies},
         "attention_us": attn_us,
         "roofline": {"bound": "hbm", "achieved": alg / (attn_us * 1e-6) / 1e9, "peak": hbm, "unit": "GB/s",
                      "frac": alg / (attn_us * 1e-6) / 1e9 / hbm, "algorithmic_bytes_per_launch": alg,
-                     "traffic": traffic, "kernel": "mla_decode_kernel<16,1,true>"},
+                     "traffic": traffic, "kernel": f"mla_decode_kernel<{S * H},{S},true>"},
         "gpu_launches": 3 * args.steps,
     }
     if acc is not None:

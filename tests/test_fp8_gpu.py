@@ -62,11 +62,12 @@ def test_fp8_tail_codes_never_reach_the_result(dev, orc):
     compare(g_out, g_lse, r_out, r_lse, what="fp8 NaN tails")
 
 
-def test_fp8_widening_is_exact_for_every_code(dev):
+def test_fp8_every_code_reaches_the_output_exactly(dev):
     # One visible token with scale 1: its weight is 1, so each output row is
-    # the token's 512 value columns as widened by the kernel.  The row holds
-    # every code but the two NaN patterns s|1111|111, twice (subnormals and
-    # both zeros included), checked against torch's float8_e4m3fn decoding.
+    # the token's 512 value columns as the output MMA reads them (the codes
+    # themselves, weight 1 exactly in e4m3).  The row holds every code but the
+    # two NaN patterns s|1111|111, twice (subnormals and both zeros included),
+    # checked against torch's float8_e4m3fn decoding.
     inp = mi.small(B=1, s_q=1, H=16, seqlens=[1], seed=68)
     cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=69)
     finite = torch.tensor([c for c in range(256) if c & 0x7F != 0x7F] + [0x38, 0xB8])
