@@ -913,21 +913,27 @@ __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const 
             if (!(ok = warp_wait(sm.bar(kBarPFull + pb), pu & 1, sm.abort_flag, p.err))) break;
             ptx::tc_fence_after();
             const uint32_t pa = sm.p + pb * 2 * C::QCHUNK;
-#pragma unroll 1
+            uint32_t a0[4];
+#pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t u = cc + j;
                 const int slot = static_cast<int>(u % R);
                 // landed long ago (the score MMA read it); waited on for the ordering
-                if (!(ok = warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err))) break;
-                ptx::tc_fence_after();
-                const uint32_t a0 = sm.slot(slot);
-#pragma unroll 1
-                for (int kk = 0; kk < 4; ++kk)
-                    ptx::mma_e4m3_ss_elect(tmem + j * 2 * N, ptx::desc_sw128(a0 + 4096u * kk, 8192, 1024),
-                                           ptx::desc_sw128(pa + 32u * kk, 16, 1024), idO, (t != tb) || kk != 0);
-                ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
+                ok = ok && warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err);
+                a0[j] = sm.slot(slot);
             }
             if (!ok) break;
+            ptx::tc_fence_after();
+            // consecutive instructions go to different O^T blocks
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    ptx::mma_e4m3_ss_elect(tmem + j * 2 * N, ptx::desc_sw128(a0[j] + 4096u * kk, 8192, 1024),
+                                           ptx::desc_sw128(pa + 32u * kk, 16, 1024), idO, (t != tb) || kk != 0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                ptx::mma_commit_elect(sm.bar(kBarEmpty + static_cast<int>((cc + j) % R)));
             ptx::mma_commit_elect(sm.bar(kBarPEmpty + pb));
             cc += kF8Units;
             ++it;

@@ -84,6 +84,22 @@ def test_fp8_every_code_reaches_the_output_exactly(dev):
         np.testing.assert_array_equal(g_out[0, 0, h], expect)
 
 
+@pytest.mark.parametrize("H,s_q", [(16, 1), (16, 2)])
+def test_fp8_negative_and_zero_scales(dev, orc, H, s_q):
+    # a token's scale may be any fp32 value: negative scales negate the row,
+    # zero scales zero it (its score is 0, its value the zero vector)
+    inp = mi.small(B=3, s_q=s_q, H=H, seqlens=[300, 777, 64], seed=74)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=75)
+    g = torch.Generator().manual_seed(76)
+    sign = torch.randint(0, 3, cache.scale.shape, generator=g)  # 0: negate, 1: zero, 2: keep
+    cache.scale = torch.where(sign == 0, -cache.scale, torch.where(sign == 1, torch.zeros_like(cache.scale),
+                                                                   cache.scale))
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err == 0
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"fp8 signed scales s_q={s_q}")
+
+
 def test_fp8_paging_invariance(dev):
     # the same logical rows through an identity and a shuffled table: bitwise equal
     a = mi.small(B=2, s_q=1, H=16, seqlens=[300, 900], table="identity", seed=64)
