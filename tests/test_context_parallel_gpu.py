@@ -12,7 +12,7 @@ import torch
 import decode_attention_latent_b200 as mla
 import mla_inputs as mi
 import oracle
-from decode_attention_latent_b200.context_parallel import decode_context_parallel, local_shard
+from decode_attention_latent_b200.context_parallel import decode_context_parallel, decode_local_state, local_shard
 from test_parity import compare, ulp_bf16
 
 pytestmark = pytest.mark.gpu
@@ -50,19 +50,23 @@ def test_merge_states_matches_oracle(dev, orc, W, rows):
     assert np.abs(g_lse[fin] - r_lse[fin]).max() <= 1e-5
 
 
-@pytest.mark.parametrize("H,W", [(16, 2), (16, 3), (16, 8), (128, 2)])
-def test_emulated_ranks_match_oracle(dev, orc, H, W):
-    inp = mi.small(B=3, s_q=1, H=H, seqlens=[1, 700, 64 * 20 + 5], seed=51)
+@pytest.mark.parametrize("H,W,s_q", [(16, 2, 1), (16, 3, 1), (16, 8, 1), (128, 2, 1),
+                                     (16, 2, 2), (16, 3, 4), (32, 3, 2), (16, 8, 8), (64, 2, 2)])
+def test_emulated_ranks_match_oracle(dev, orc, H, W, s_q):
+    # lengths below s_q - 1, at page edges and long; every rank's state from
+    # decode_local_state (the causal query on the last rank, folded before it)
+    inp = mi.small(B=5, s_q=s_q, H=H, seqlens=[1, 66, 129, 700, 64 * 20 + 5], seed=51)
     q, kv = inp.q.to(dev), inp.kv_cache.to(dev)
     outs, lses = [], []
     for r in range(W):
-        sl, bt = local_shard(inp.cache_seqlens, inp.block_table, W, r)
-        o, l = mla.decode(q, kv, bt.to(dev), sl.to(dev), inp.scale)
+        sl, bt = local_shard(inp.cache_seqlens, inp.block_table, W, r, s_q)
+        o, l = decode_local_state(q, kv, bt.to(dev), sl.to(dev), inp.scale, r == W - 1)
         outs.append(o)
         lses.append(l)
     out, lse = mla.merge_states(torch.stack(outs), torch.stack(lses))
     r_out, r_lse = orc.direct(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.scale)
-    compare(out.float().cpu().numpy(), lse.cpu().numpy(), r_out, r_lse, what=f"context-parallel W={W}")
+    compare(out.float().cpu().numpy(), lse.cpu().numpy(), r_out, r_lse,
+            what=f"context-parallel W={W} s_q={s_q} H={H}")
 
 
 def test_one_rank_nccl_group_is_plain_decode(dev):
@@ -83,8 +87,9 @@ def test_one_rank_nccl_group_is_plain_decode(dev):
     assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
 
 
-def test_multi_token_query_is_refused(dev):
-    inp = mi.small(B=1, s_q=2, H=16, seqlens=[100], seed=53)
+def test_too_many_query_columns_are_refused(dev):
+    # s_q > 1 folds the positions into heads before the last rank: s_q H <= 128
+    inp = mi.small(B=1, s_q=2, H=128, seqlens=[100], seed=53)
     with pytest.raises(ValueError):
         decode_context_parallel(inp.q.to(dev), inp.kv_cache.to(dev), inp.block_table.to(dev),
                                 inp.cache_seqlens.to(dev), inp.scale)
