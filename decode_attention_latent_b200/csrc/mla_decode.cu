@@ -86,18 +86,25 @@ constexpr int kBarVtFull = kBarPEmpty + 2;         // [kMaxVt] V^T block written
 constexpr int kBarVtEmpty = kBarVtFull + kMaxVt;   // [kMaxVt] output MMA of that V^T block complete
 constexpr int kBarDrain = kBarVtEmpty + kMaxVt;
 constexpr int kBarDrainO = kBarDrain + 1;
-// FP8 cache (16 query columns).  The tensor cores read the e4m3 codes as
-// they lie in the cache (tcgen05.mma kind::f8f6f4): the ring's slots are 16 KB
-// "units", one 128-column group of a tile (128 rows x 128 bytes of codes, both
-// pages, 128-byte swizzled), five per tile, the last holding the 64 rope
-// columns and the zero fill of its TMA box.  The score MMA reads a unit
-// K-major (rows = tokens); the output MMA reads latent units 0-3 again,
-// MN-major (rows = tokens, the 128 latent dims contiguous), as V^T.  The
-// tile's 128 token scales land with its first unit in a ring of 512-byte
-// buffers after the slot ring.
+// FP8 cache (16 or 32 query columns).  The tensor cores read the e4m3 codes
+// as they lie in the cache (tcgen05.mma kind::f8f6f4): the ring's slots are
+// 16 KB "units", one 128-column group of a tile (128 rows x 128 bytes of
+// codes, both pages, 128-byte swizzled), five per tile, the last holding the
+// 64 rope columns and the zero fill of its TMA box.  The score MMA reads a
+// unit K-major (rows = tokens) and frees it.  A second producer loads the
+// tile's four latent units again -- from L2, just read -- into a V ring of
+// kF8VRing units after the first, where the output MMA reads them MN-major
+// (rows = tokens, the 128 latent dims contiguous) as V^T.  The tile's 128
+// token scales land with its first unit in a ring of 512-byte buffers after
+// the V ring.
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
 constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
 constexpr uint32_t kF8UnitBytes = 16384;   // one ring slot: a unit's codes
+template <int N>
+__host__ __device__ constexpr int f8_vring()  // V-ring units: one tile's four and one more at 16 columns
+{
+    return N == 16 ? 5 : 4;
+}
 // Token scales of tile T are replaced by tile T + 8's once the slot of unit
 // 5 (T + 8) - R is free: for R <= 16 a unit of tile T + 5 or later, freed only
 // after the softmax of tile T has read them.
@@ -119,10 +126,13 @@ constexpr float kTau8 = 8.f;
 // entry for "q split written".
 constexpr int kBarF8Full = kBarDrainO + 1;
 constexpr int kBarQsFull = kBarF8Full;
+constexpr int kBarVFull = kBarF8Full + 1;          // [f8_vring] a V-ring unit landed
+constexpr int kBarVEmpty = kBarF8Full + 8;         // [f8_vring] the output MMA has read it
 constexpr int kScBufs = 4;
 constexpr uint32_t kScBytes = kScBufs * 128 * 4;   // (unused; kept for the layout of the bf16 instances)
 constexpr uint32_t kQScaleBytes = 128;              // FP8: the per-row q scales
 constexpr int kBarF8Reserved = kBarF8Full + 8 + 2 * kScBufs;
+static_assert(kBarVFull + 5 <= kBarVEmpty && kBarVEmpty + 5 <= kBarF8Reserved, "FP8 V-ring barriers");
 constexpr int kNumBars = kBarF8Reserved;
 // The reduction buffers after the barriers are read as float4: keep them
 // 16-byte aligned (rounded to 128 B).
@@ -836,9 +846,8 @@ __device__ void output_mma_warp(const DecodeParams &p, const Range &w, const Sme
 // Score MMA: S^T(t) = sum over the tile's five units of K_unit q_unit^T, with
 // q as its two e4m3 terms stacked as 2N rows (hi rows 0..N-1, lo rows N..2N-1,
 // so S^T has 2N columns whose halves the softmax adds), K = 32 codes per
-// instruction.  Latent
-// units stay in the ring for the output MMA; the rope unit is free after the
-// score MMA (both of its slot's arrivals come from here).
+// instruction.  Every unit's slot is free once its instructions complete (the
+// output MMA reads its own copy of the latent units from the V ring).
 template <int N, int SQ>
 __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
@@ -877,7 +886,6 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
                     ptx::mma_e4m3_ss_elect(d, ptx::desc_sw128(a0 + 32u * kk, 16, 1024),
                                            ptx::desc_sw128(q0 + 32u * kk, 16, 1024), idS, (k | kk) != 0);
                 ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
-                if (k == kF8Units - 1) ptx::mma_commit_elect(sm.bar(kBarEmpty + slot));
             }
             if (!ok) break;
             ptx::mma_commit_elect(sm.bar(kBarSFull + sb));
@@ -891,17 +899,18 @@ __device__ void score_mma_warp_f8(const DecodeParams &p, const Range &w, const S
 }
 
 // Output MMA: O^T block j += V^T_j P~^T, V^T_j = latent unit j of the tile read
-// MN-major straight from its ring slot, P~ the weights as two e4m3 terms
-// stacked as 2N rows of 128 tokens (K-major), 32 tokens per instruction; the
-// epilogue adds the block's two column halves.  Each unit's slot is free once
-// its MMAs are complete.
+// MN-major from its V-ring slot, P~ the weights as two e4m3 terms stacked as
+// 2N rows of 128 tokens (K-major), 32 tokens per instruction; the epilogue
+// adds the block's two column halves.  Each V-ring slot is free once its
+// instructions complete.
 template <int N, int SQ>
 __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const Smem &sm, uint32_t tmem)
 {
     using C = Cfg<N, SQ>;
     constexpr uint32_t idO = ptx::idesc_e4m3_f32(128, 2 * N, true, false);  // V^T MN-major, P~^T K-major
-    const uint32_t R = static_cast<uint32_t>(p.ring);
-    uint32_t it = 0, cc = 0;
+    constexpr uint32_t RV = f8_vring<N>();
+    const uint32_t vbase = sm.ring + static_cast<uint32_t>(p.ring) * kF8UnitBytes;
+    uint32_t it = 0, vc = 0;
     bool ok = true;
     for (int b = w.b0; b <= w.b1 && ok; ++b) {
         const int L = max(0, __ldg(p.seqlens + b));
@@ -916,11 +925,10 @@ __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const 
             uint32_t a0[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t u = cc + j;
-                const int slot = static_cast<int>(u % R);
-                // landed long ago (the score MMA read it); waited on for the ordering
-                ok = ok && warp_wait(sm.bar(kBarFull + slot), (u / R) & 1, sm.abort_flag, p.err);
-                a0[j] = sm.slot(slot);
+                const uint32_t v = vc + j;
+                const int slot = static_cast<int>(v % RV);
+                ok = ok && warp_wait(sm.bar(kBarVFull + slot), (v / RV) & 1, sm.abort_flag, p.err);
+                a0[j] = vbase + slot * kF8UnitBytes;
             }
             if (!ok) break;
             ptx::tc_fence_after();
@@ -932,15 +940,75 @@ __device__ void output_mma_warp_f8(const DecodeParams &p, const Range &w, const 
                     ptx::mma_e4m3_ss_elect(tmem + j * 2 * N, ptx::desc_sw128(a0[j] + 4096u * kk, 8192, 1024),
                                            ptx::desc_sw128(pa + 32u * kk, 16, 1024), idO, (t != tb) || kk != 0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                ptx::mma_commit_elect(sm.bar(kBarEmpty + static_cast<int>((cc + j) % R)));
+            for (int j = 0; j < 4; ++j) ptx::mma_commit_elect(sm.bar(kBarVEmpty + static_cast<int>((vc + j) % RV)));
             ptx::mma_commit_elect(sm.bar(kBarPEmpty + pb));
-            cc += kF8Units;
+            vc += 4;
             ++it;
         }
     }
     ptx::mma_commit_elect(sm.bar(kBarDrainO));
     warp_wait(sm.bar(kBarDrainO), 0, sm.abort_flag, p.err, false);
+}
+
+// FP8 cache: the V producer (the first transposer warp, idle otherwise).
+// Walks the same ranges, tiles and page-table windows as the producer and
+// loads each tile's four latent units again into the V ring; the producer's
+// load of the same bytes has normally just brought them into L2, so the HBM
+// traffic stays one read.
+template <int N, int SQ>
+__device__ void v_producer_warp(const DecodeParams &p, const Range &w, const Smem &sm, const CUtensorMap *kv_map)
+{
+    constexpr uint32_t RV = f8_vring<N>();
+    const int lane = threadIdx.x & 31;
+    const uint32_t vbase = sm.ring + static_cast<uint32_t>(p.ring) * kF8UnitBytes;
+    uint32_t vc = 0;  // V-ring slot uses so far
+    bool ok = true;
+    for (int b = w.b0; b <= w.b1 && ok; ++b) {
+        const int tb = (b == w.b0) ? w.t0 : 0;
+        const int32_t *bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks;
+        int win = 2 * tb;
+        const int raw_cur = table_entry(bt, win, p, lane);
+        const int raw_nxt = table_entry(bt, win + 32, p, lane);
+        const int L = max(0, __ldg(p.seqlens + b));
+        const int nt = tiles_of(L);
+        const int te = min((b == w.b1) ? w.t1 : nt, nt);
+        if (tb >= te) continue;
+        const int npages = (L + kPage - 1) / kPage;
+        int cur = checked_page(raw_cur, win, npages, p, lane);
+        int nxt = checked_page(raw_nxt, win + 32, npages, p, lane);
+        for (int t = tb; t < te && ok; ++t) {
+            if (2 * t >= win + 32) {
+                win += 32;
+                cur = nxt;
+                nxt = load_pages(bt, win + 32, npages, p, lane);
+            }
+            const int phys0 = __shfl_sync(0xffffffffu, cur, 2 * t - win);
+            const int phys1 = __shfl_sync(0xffffffffu, cur, 2 * t + 1 - win);
+            const bool live1 = (t * kTile + kPage) < L;
+            const uint32_t b8 = live1 ? 2 * kF8Half : kF8Half;
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t v = vc + j;
+                const int slot = static_cast<int>(v % RV);
+                if (!warp_wait(sm.bar(kBarVEmpty + slot), ((v / RV) & 1) ^ 1, sm.abort_flag, p.err)) {
+                    ok = false;
+                    vc += j;
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx_elect(sm.bar(kBarVFull + slot), b8);
+                const uint32_t dst = vbase + slot * kF8UnitBytes;
+                ptx::tma_load_3d_elect(dst, kv_map, sm.bar(kBarVFull + slot), 128 * j, 0, phys0);
+                if (live1) ptx::tma_load_3d_elect(dst + kF8Half, kv_map, sm.bar(kBarVFull + slot), 128 * j, 0, phys1);
+            }
+            if (ok) vc += 4;
+        }
+    }
+    if (!ok) {
+        // Let every load this warp issued land before the CTA exits.
+        const uint32_t first = vc > RV ? vc - RV : 0;
+        for (uint32_t v = first; v < vc; ++v)
+            warp_wait(sm.bar(kBarVFull + static_cast<int>(v % RV)), (v / RV) & 1, sm.abort_flag, p.err, false);
+    }
 }
 
 // -- transposer: 4 warps copy V(t) into the TMEM ring as V^T ----------------
@@ -1437,16 +1505,23 @@ __device__ void softmax_warps(const DecodeParams &p, const Range &w, int g, cons
                 // Rows past the sequence's end in its last tile hold whatever the
                 // cache (or an earlier unit) left there, NaN codes included; their
                 // weights are zero, and the V^T the output MMA reads must be finite
-                // too: this thread zeroes its row of the tile's four latent units.
-                const int valid = L - t * kTile;
-                const int r = 32 * wq + lane;
-                if (valid < kTile && r >= valid) {
-                    const uint32_t R = static_cast<uint32_t>(p.ring);
+                // too: once the tile's four V-ring units have landed, this thread
+                // zeroes its row of them.
+                const int valid = L - t * kTile;  // the same in every thread
+                if (valid < kTile) {
+                    constexpr uint32_t RV = f8_vring<N>();
+                    const uint32_t vbase = sm.ring + static_cast<uint32_t>(p.ring) * kF8UnitBytes;
+                    const int r = 32 * wq + lane;
 #pragma unroll 1
                     for (int j = 0; j < 4; ++j) {
-                        const uint32_t ra = sm.slot(static_cast<int>((kF8Units * it + j) % R)) + r * 128u;
+                        const uint32_t v = 4 * it + j;
+                        const int slot = static_cast<int>(v % RV);
+                        wait_ok = warp_wait(sm.bar(kBarVFull + slot), (v / RV) & 1, sm.abort_flag, p.err) && wait_ok;
+                        if (r >= valid) {
+                            const uint32_t ra = vbase + slot * kF8UnitBytes + r * 128u;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) ptx::st_shared_v4(ra + 16u * c, 0u, 0u, 0u, 0u);
+                            for (int c = 0; c < 8; ++c) ptx::st_shared_v4(ra + 16u * c, 0u, 0u, 0u, 0u);
+                        }
                     }
                 }
             } else {
@@ -1510,7 +1585,8 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     sm.ring = base;
     sm.slot_bytes = F8 ? kF8UnitBytes : C::SLOT_BYTES;
     uint32_t off = p.ring * (F8 ? kF8UnitBytes : C::SLOT_BYTES);
-    sm.f8 = base + off;  // FP8: the ring of units, the token scales, then q (split in place) and P~^T
+    if constexpr (F8) off += f8_vring<N>() * kF8UnitBytes;
+    sm.f8 = base + off;  // FP8: the unit ring, the V ring, the token scales, then q (split in place) and P~^T
     if constexpr (F8) off += kRawScBytes;
     sm.q = base + off;
     constexpr uint32_t qreg = F8 ? C::QS8 : C::QBYTES;
@@ -1530,12 +1606,15 @@ __device__ __forceinline__ bool decode_setup(const DecodeParams &p, const CUtens
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ring; ++s) {
             ptx::mbar_init(sm.bar(kBarFull + s), 1);
-            // FP8: a unit's slot is free after the score and the output MMA
-            // (the rope unit: two commits of the score MMA)
-            ptx::mbar_init(sm.bar(kBarEmpty + s), F8 ? 2 : C::EMPTY_ARRIVALS);
+            // FP8: a unit's slot is free after the score MMA
+            ptx::mbar_init(sm.bar(kBarEmpty + s), F8 ? 1 : C::EMPTY_ARRIVALS);
         }
         if constexpr (F8) {
             ptx::mbar_init(sm.bar(kBarQsFull), 4);  // one arrival per softmax warp
+            for (int i = 0; i < f8_vring<N>(); ++i) {
+                ptx::mbar_init(sm.bar(kBarVFull + i), 1);
+                ptx::mbar_init(sm.bar(kBarVEmpty + i), 1);
+            }
         } else {
             // (unused by the bf16 instances; kept so their set-up is unchanged)
             for (int i = 0; i < 4; ++i) {
@@ -1631,7 +1710,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_const
         } else if (warp < 6) {
             softmax_warps<N, SQ, F8>(p, w, g, sm, tmem);
         } else if (warp < 10) {
-            transposer_warps<N, SQ, F8>(p, w, sm, tmem);
+            if constexpr (F8) {
+                if (warp == 6) v_producer_warp<N, SQ>(p, w, sm, &kv_map);
+            } else {
+                transposer_warps<N, SQ, F8>(p, w, sm, tmem);
+            }
         } else {
             if constexpr (F8) output_mma_warp_f8<N, SQ>(p, w, sm, tmem);
             else output_mma_warp<N, SQ>(p, w, sm, tmem);
@@ -1917,7 +2000,7 @@ int ring_for(int smem_optin, size_t *smem_bytes)
 {
     using C = Cfg<N, SQ>;
     const int fixed = static_cast<int>((F8 ? C::QS8 : C::QBYTES) + C::PBYTES + misc_bytes<N>() + 1024 +
-                                       (F8 ? kRawScBytes + kQScaleBytes : 0));
+                                       (F8 ? kRawScBytes + kQScaleBytes + f8_vring<N>() * kF8UnitBytes : 0));
     const uint32_t slot = F8 ? kF8UnitBytes : C::SLOT_BYTES;
     int R = (smem_optin - fixed) / static_cast<int>(slot);
     if (R > kMaxRing) R = kMaxRing;
