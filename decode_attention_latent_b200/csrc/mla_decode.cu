@@ -35,6 +35,13 @@
 // it, so the slot ring never waits on the softmax, and a V^T block is released
 // as soon as its output MMAs complete.  Warps: producer, score MMA, 4 softmax,
 // 4 transposer, output MMA.
+//
+// The FP8 instances (an e4m3 cache with one fp32 scale per token) feed the
+// codes to the tensor cores as they land (kind::f8f6f4): the score MMA reads
+// each 128-column unit K-major against q written as two e4m3 terms, the
+// softmax writes its weights as two e4m3 terms, and the output MMA reads V^T
+// MN-major from a second copy of the latent units that one of the transposer
+// warps loads into a V ring (the other three are idle there).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -106,8 +113,9 @@ __host__ __device__ constexpr int f8_vring()  // V-ring units: one tile's four a
     return N == 16 ? 5 : 4;
 }
 // Token scales of tile T are replaced by tile T + 8's once the slot of unit
-// 5 (T + 8) - R is free: for R <= 16 a unit of tile T + 5 or later, freed only
-// after the softmax of tile T has read them.
+// 5 (T + 8) - R is free: for R <= 16 a unit of tile T + 4 or later, freed by
+// the score MMA of that tile, which waits for the softmax of tile T + 2 to
+// have read its S^T buffer -- after the softmax of tile T read the scales.
 constexpr int kRawScBufs = 8;
 constexpr uint32_t kRawScBytes = kRawScBufs * 512;
 // q split into two e4m3 terms per element (see softmax_warps): per unit a hi
@@ -493,8 +501,8 @@ struct Cfg {
 struct Smem {
     uint32_t ring, q, p;     // shared-window addresses: slot ring, Q, P^T buffers
     uint32_t slot_bytes;     // bytes per ring slot
-    uint32_t f8;             // shared-window address of the FP8 staging ring (FP8 cache only)
-    float *tscale;           // FP8: token scales of kScBufs tiles [kScBufs][128]
+    uint32_t f8;             // shared-window address of the FP8 token-scale buffers (FP8 cache only)
+    float *tscale;           // FP8: the per-row q scales 2^-a_n [N]
     uint32_t bars;           // address of barrier 0
     float *red, *lred;       // column-max exchange [4][N], sum exchange [4][N]
     float *mu, *shift;       // reference max [N], its last shift [N]
@@ -1688,7 +1696,7 @@ __device__ __forceinline__ void decode_teardown(uint32_t tmem)
 }
 
 // Warps: 0 producer, 1 score MMA (and TMEM owner), 2-5 softmax + epilogue,
-// 6-9 transposer, 10 output MMA.
+// 6-9 transposer (FP8: 6 the V producer, 7-9 idle), 10 output MMA.
 template <int N, int SQ, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
