@@ -145,6 +145,34 @@ def test_fp8_last_token_seen_by_the_second_query_position(dev, orc):
     compare(g_out, g_lse, r_out, r_lse, what="fp8 s_q=2 last token")
 
 
+@pytest.mark.parametrize("name", ["b8_h16_l64k", "b32_sq2_h16_l16k_outliers"])
+def test_fp8_full_size_workload(dev, orc, name):
+    # the launch configuration `bench.py --fp8` times (metadata, attention and
+    # combine over every SM), on its inputs at full size; every sequence checked
+    inp = mi.make_inputs(mi.WORKLOADS[name], seed=0)
+    nb = inp.kv_cache.shape[0]
+    inp.kv_cache = None
+    cache = mi.fp8_cache(nb, seed=1)
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err == 0
+    r_out, r_lse = orc.direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table, inp.cache_seqlens, inp.scale)
+    compare(g_out, g_lse, r_out, r_lse, what=f"fp8 {name}")
+
+
+@pytest.mark.parametrize("H,s_q", [(16, 1), (16, 2)])
+def test_fp8_bad_block_table_sets_error_word(dev, orc, H, s_q):
+    # an entry naming no block of the cache: both loads of its tile read
+    # block 0 instead, the error word says so, and the other sequence is exact
+    inp = mi.small(B=2, s_q=s_q, H=H, seqlens=[300, 200], seed=74)
+    cache = mi.fp8_cache(inp.kv_cache.shape[0], seed=75)
+    good = inp.block_table[0:1].clone()
+    inp.block_table[1, 2] = inp.kv_cache.shape[0] + 5
+    g_out, g_lse, err = run_fp8(inp, cache, dev)
+    assert err & mla.DEVERR_BLOCK_TABLE
+    r_out, r_lse = orc.direct_fp8(inp.q[0:1], cache.codes, cache.scale, good, inp.cache_seqlens[0:1], inp.scale)
+    compare(g_out[0:1], g_lse[0:1], r_out, r_lse, what=f"fp8 bad page, other sequence (s_q={s_q})")
+
+
 @pytest.mark.parametrize("H,s_q", [(64, 1), (32, 2), (16, 4), (128, 1)])
 def test_fp8_unsupported_shape_is_refused(dev, H, s_q):
     inp = mi.small(B=1, s_q=s_q, H=H, seqlens=[100], seed=66)

@@ -51,6 +51,21 @@ def test_naive_matches_oracle(dev, orc, s_q, H, lens, n_sms):
     compare(g_out, g_lse, r_out, r_lse, what=f"naive s_q={s_q} H={H}")
 
 
+def test_naive_full_size_workload(dev, orc):
+    # the launch configuration `bench.py --naive` times: the 64K-context,
+    # 16-head workload at full size over every SM; the oracle checks two
+    # whole sequences (its per-token decompression makes all eight slow)
+    w = mi.WORKLOADS["b8_h16_l64k"]
+    base = mi.make_inputs(w, seed=0)
+    nv = mi.naive_inputs(w.B, w.s_q, w.H, seed=1)
+    g_out, g_lse, err = run_naive(base, nv, dev)
+    assert err == 0
+    seqs = [0, 5]
+    r_out, r_lse = orc.naive(nv.q, base.kv_cache, nv.w_uk, nv.w_uv, base.block_table, base.cache_seqlens,
+                             base.scale, seqs=seqs)
+    compare(g_out, g_lse, r_out, r_lse, seqs=seqs, what="naive b8_h16_l64k")
+
+
 def test_naive_page_table_invariance(dev):
     """The same logical rows through an identity and a shuffled table give
     bitwise equal results (integer page indexing is exact)."""
