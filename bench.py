@@ -724,6 +724,9 @@ def run_fp8(args):
         r_out, r_lse = oracle.default().direct_fp8(inp.q, cache.codes, cache.scale, inp.block_table,
                                                    inp.cache_seqlens, inp.scale)
         acc = accuracy(out.float().cpu().numpy(), lse.cpu().numpy(), r_out, r_lse, None, B)
+    sampler = ClockSampler(0).start()
+    time.sleep(0.3)
+    t_start = time.time()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for k in range(args.steps):
         ev[k][0].record(); call(k); ev[k][1].record()
@@ -735,6 +738,7 @@ def run_fp8(args):
     for k in range(args.steps):
         ea[k][0].record(); decode(k, lib.mla_decode_attention_fp8); ea[k][1].record()
     torch.cuda.synchronize(dev)
+    clocks = sampler.stop(t_start, time.time())
     assert mla.get_device_error(sched) == 0
     attn_us = statistics.mean(a.elapsed_time(b) for a, b in ea) * 1e3
     tokens = int(inp.cache_seqlens.sum())
@@ -760,6 +764,7 @@ def run_fp8(args):
                      "frac": alg / (attn_us * 1e-6) / 1e9 / hbm, "algorithmic_bytes_per_launch": alg,
                      "traffic": traffic, "kernel": f"mla_decode_kernel<{S * H},{S},true>"},
         "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
     }
     if acc is not None:
         line["accuracy"] = acc
