@@ -100,10 +100,10 @@ constexpr int kBarDrainO = kBarDrain + 1;
 // 64 rope columns and the zero fill of its TMA box.  The score MMA reads a
 // unit K-major (rows = tokens) and frees it.  A second producer loads the
 // tile's four latent units again -- from L2, just read -- into a V ring of
-// kF8VRing units after the first, where the output MMA reads them MN-major
-// (rows = tokens, the 128 latent dims contiguous) as V^T.  The tile's 128
-// token scales land with its first unit in a ring of 512-byte buffers after
-// the V ring.
+// f8_vring() units after the unit ring, where the output MMA reads them
+// MN-major (rows = tokens, the 128 latent dims contiguous) as V^T.  The
+// tile's 128 token scales land with its first unit in a ring of 512-byte
+// buffers after the V ring.
 constexpr int kF8Units = 5;                // per tile: latent columns 0-511 in 4 groups, then the rope group
 constexpr uint32_t kF8Half = 8192;         // one page's 64 rows x 128 B of codes
 constexpr uint32_t kF8UnitBytes = 16384;   // one ring slot: a unit's codes
