@@ -125,10 +125,12 @@ constexpr uint32_t kRawScBytes = kRawScBufs * 512;
 // FP8 weights: the reference max sits kLift8 below the largest log2 weight
 // seen when it last moved, so weights reach 2^kLift8 and stay above e4m3's
 // subnormal range (2^-6) down to 2^-13 of the largest; it moves again when a
-// weight would pass 2^kTau8 (e4m3 holds up to 448).  l and lse use the same
-// reference, so the result does not depend on it.
+// weight would pass 2^kTau8 = 430 (e4m3 holds up to 448 = 2^8.81; each move
+// rescales O^T after waiting for the previous tile's output MMA, and 2^8.75
+// rather than 2^8 made that 1.5 us per call rarer on both FP8 workloads).  l
+// and lse use the same reference, so the result does not depend on it.
 constexpr float kLift8 = 7.f;
-constexpr float kTau8 = 8.f;
+constexpr float kTau8 = 8.75f;
 // The barrier block below keeps the layout of an earlier design (the bf16
 // instances are laid out exactly as before); the FP8 instance uses its first
 // entry for "q split written".
